@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""WAITS prefill score + select + compact throughput on B200.
+
+Workload: the Llama-3.1-8B-shaped stack -- 32 layers with independently
+seeded bf16 Q/K/V (sink + 64 heavy hitters per KV head), batch 1, N=32768,
+32 query / 8 KV heads, d=128, a=1, b=16, R=16, B=2048 (``--budget``).
+A step runs score -> select -> compact once for every layer, through the C
+ABI (waits_score, waits_select, waits_compact on one stream).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank owns its own 32-layer
+stack (weak scaling); there is no data-path collective.  Prints one JSON
+line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from prefill_eviction_scoring_b200 import _lib, api  # noqa: E402
+from prefill_eviction_scoring_b200 import workloads as wl  # noqa: E402
+
+METRIC = "prompt tokens/s scored+compacted per layer (8B shape, N=32K); % of roofline"
+UNIT = "tokens/s"
+CONFIG = "llama8b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1590.0}
+KERNELS_PER_LAYER = 5   # plan, pass 1, pass 2, select, compact
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--budget", type=int, default=2048)
+    p.add_argument("--layers", type=int, default=wl.CONFIGS[CONFIG].layers)
+    p.add_argument("--e2e-layers", type=int, default=4)
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------ arithmetic ---
+def first_active_row(N, a, b):
+    """First row with non-zero fp32 forgetting-curve weight (the predicate
+    the library's planner uses), by numpy float32."""
+    if a == 0.0:
+        return 0
+    q = np.arange(N)
+    c = np.float32(N) - np.float32(b) - np.float32(0.5)
+    with np.errstate(over="ignore"):
+        w = np.float32(1.0) / (np.float32(1.0) + np.exp(np.float32(-a) * (q.astype(np.float32) - c)))
+    nz = np.nonzero(w != 0)[0]
+    return int(nz[0]) if len(nz) else N
+
+
+def scorer_flops(lens, Hq, d, a, b):
+    """Algorithmic tensor FLOPs of one scorer call: two passes of causal
+    QK^T over the active rows, 2*d FLOPs per logit."""
+    logits = 0
+    for N in lens:
+        q0 = first_active_row(N, a, b)
+        logits += (N * (N + 1) - q0 * (q0 + 1)) // 2     # sum_{q=q0}^{N-1} (q+1)
+    return 2 * 2 * d * Hq * logits, logits * Hq
+
+
+def select_compact_bytes(lens, Hkv, d, B):
+    """Algorithmic HBM bytes: scores read by select, idx written; compaction
+    reads and writes min(B, N) rows of K and of V per KV head."""
+    T = sum(lens)
+    sel = Hkv * T * 4 + len(lens) * Hkv * B * 4
+    rows = sum(min(B, N) for N in lens) * Hkv
+    comp = 2 * 2 * rows * d * 2 + len(lens) * Hkv * B * 4
+    return sel, comp
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return m, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------- plumbing ---
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self):
+        torch.cuda.set_device(self.local)
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        torch.cuda.synchronize()
+        if self.pg:
+            self.pg.barrier()
+        torch.cuda.synchronize()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, local_rank):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        self.gpu = ids[local_rank] if local_rank < len(ids) else str(local_rank)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons, power = [], [], set(), []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_median": statistics.median(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+class LayerCall:
+    """Preallocated buffers for one layer and the three C-ABI calls."""
+
+    def __init__(self, lay, B, shape, workspace, ws_bytes):
+        self.lay = lay
+        T, Hq, d = lay.Q.shape
+        Hkv = lay.K.shape[1]
+        dev = lay.Q.device
+        self.shape = shape
+        self.ws, self.ws_bytes = workspace, ws_bytes
+        self.scores = torch.empty((Hkv, T), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((1, Hkv, B), dtype=torch.int32, device=dev)
+        self.kept = torch.empty((1,), dtype=torch.int32, device=dev)
+        self.Ko = torch.empty((1, Hkv, B, d), dtype=torch.bfloat16, device=dev)
+        self.Vo = torch.empty_like(self.Ko)
+        self.B = B
+
+    def score(self, lib, a, b, stream):
+        return lib.waits_score(ctypes.byref(self.shape), self.lay.Q.data_ptr(),
+                               self.lay.K.data_ptr(), a, b, self.scores.data_ptr(),
+                               self.ws.data_ptr(), self.ws_bytes, stream)
+
+    def select(self, lib, R, stream):
+        return lib.waits_select(ctypes.byref(self.shape), self.scores.data_ptr(), R, self.B,
+                                self.idx.data_ptr(), self.kept.data_ptr(), self.ws.data_ptr(),
+                                self.ws_bytes, stream)
+
+    def compact(self, lib, stream):
+        return lib.waits_compact(ctypes.byref(self.shape), self.lay.K.data_ptr(),
+                                 self.lay.V.data_ptr(), self.idx.data_ptr(), self.kept.data_ptr(),
+                                 self.B, self.Ko.data_ptr(), self.Vo.data_ptr(),
+                                 self.ws.data_ptr(), self.ws_bytes, stream)
+
+
+def cpu_oracle_sample(lay, a, b, R, B, g=0):
+    """Time the fp64 oracle on KV head g of one layer (its G query heads):
+    score, select and compact.  Returns (seconds, threads)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    Hq, Hkv = lay.Q.shape[1], lay.K.shape[1]
+    G = Hq // Hkv
+    Qn = wl.to_numpy64(lay.Q[:, g * G:(g + 1) * G])
+    Kn = wl.to_numpy64(lay.K[:, g:g + 1])
+    Kb, Vb = wl.to_bits(lay.K[:, g:g + 1]), wl.to_bits(lay.V[:, g:g + 1])
+    cu = lay.cu_seqlens.cpu().numpy()
+    t0 = time.perf_counter()
+    s = oracle.score(Qn, Kn, cu, a, b)
+    idx, kept = oracle.select(s, cu, R, B)
+    oracle.compact(Kb, Vb, cu, idx, kept, B)
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return dt, threads
+
+
+def config_dict(args, L, lens, spec):
+    a, b = spec.actions[0]
+    return {"workload": f"{CONFIG}: {L} layers x N={lens[0]}, Hq={spec.num_q_heads}/"
+                        f"Hkv={spec.num_kv_heads}, d={spec.head_dim}, a={a}, b={b}, "
+                        f"R={spec.recent}, B={args.budget}; sink + {spec.heavy_hitters} "
+                        f"heavy hitters per KV head",
+            "layers_per_gpu": L, "seq_len": lens[0], "batch": len(lens),
+            "num_q_heads": spec.num_q_heads, "num_kv_heads": spec.num_kv_heads,
+            "head_dim": spec.head_dim, "sigmoid_a": a, "window": b,
+            "recent_budget": spec.recent, "budget": args.budget,
+            "l2": "inputs larger than L2: each layer has its own tensors (~0.4 GB), "
+                  "a step walks all layers, so every layer starts L2-cold",
+            "parallelism": f"weak: {L}-layer stack per GPU, no collective"}
+
+
+# ------------------------------------------------------------------ ours ---
+def run_ours(args):
+    D = Dist()
+    D.init()
+    dev = torch.device("cuda", D.local)
+    lib = _lib.load()
+    spec = wl.CONFIGS[CONFIG]
+    a, b = spec.actions[0]
+    R, B, L = spec.recent, args.budget, args.layers
+    layers = [wl.make_layer(CONFIG, layer=i, device=dev)
+              for i in wl.split_layers(L, D.world, D.rank)]
+    lay0 = layers[0]
+    T, Hq, d = lay0.Q.shape
+    Hkv = lay0.K.shape[1]
+    shape = api.make_shape(lay0.cu_seqlens, T, lay0.max_seqlen, Hq, Hkv, d)
+    ws_bytes = api.workspace_bytes(shape)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    calls = [LayerCall(l, B, api.make_shape(l.cu_seqlens, T, l.max_seqlen, Hq, Hkv, d), ws,
+                       ws_bytes) for l in layers]
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+
+    def step(evs=None):
+        for i, c in enumerate(calls):
+            if evs is not None:
+                evs[i][0].record(stream)
+            _lib.check("waits_score", c.score(lib, a, b, sp))
+            if evs is not None:
+                evs[i][1].record(stream)
+            _lib.check("waits_select", c.select(lib, R, sp))
+            if evs is not None:
+                evs[i][2].record(stream)
+            _lib.check("waits_compact", c.compact(lib, sp))
+            if evs is not None:
+                evs[i][3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = ctypes.c_uint32(0)
+    _lib.check("status", lib.waits_read_device_status(ws.data_ptr(), ws_bytes, sp, ctypes.byref(st)))
+    if st.value:
+        raise RuntimeError(f"device status {st.value:#x} after warm-up")
+
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in calls]
+           for _ in range(K)]
+    t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(D.local)
+    D.barrier()
+    clocks.start()
+    t0e.record(stream)
+    for k in range(K):
+        step(evs[k])
+    t1e.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    D.barrier()
+    ms = D.max(t0e.elapsed_time(t1e)) / K
+    t_score = statistics.mean(e[0].elapsed_time(e[1]) for s_ in evs for e in s_)
+    t_sel = statistics.mean(e[1].elapsed_time(e[2]) for s_ in evs for e in s_)
+    t_comp = statistics.mean(e[2].elapsed_time(e[3]) for s_ in evs for e in s_)
+    t_score, t_sel, t_comp = D.max(t_score), D.max(t_sel), D.max(t_comp)
+
+    N = lay0.max_seqlen
+    tokens_per_step = D.world * L * sum(lay0.lens)
+    value = tokens_per_step / (ms / 1e3)
+    flops, logits = scorer_flops(lay0.lens, Hq, d, a, b)
+    sel_b, comp_b = select_compact_bytes(lay0.lens, Hkv, d, B)
+    pk, pk_kind = peaks()
+    peak_t = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
+    achieved_t = flops / (t_score / 1e3) / 1e12
+    roof = {"kernel": "scorer (waits_score: planner + pass 1 + pass 2)",
+            "bound": "tensor", "achieved": round(achieved_t, 2), "peak": peak_t,
+            "unit": "TFLOP/s", "frac": round(achieved_t / peak_t, 4), "traffic": None,
+            "peak_kind": f"bf16_tflops_sustained ({pk_kind})",
+            "flops_per_launch": flops, "launch_ms": round(t_score, 4)}
+    hbm = float(pk.get("hbm_gbs"))
+    other = [
+        {"kernel": "select", "bound": "hbm", "achieved": round(sel_b / (t_sel / 1e3) / 1e9, 1),
+         "peak": hbm, "unit": "GB/s", "frac": round(sel_b / (t_sel / 1e3) / 1e9 / hbm, 4),
+         "bytes_per_launch": sel_b, "launch_ms": round(t_sel, 4)},
+        {"kernel": "compact", "bound": "hbm",
+         "achieved": round(comp_b / (t_comp / 1e3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
+         "frac": round(comp_b / (t_comp / 1e3) / 1e9 / hbm, 4), "bytes_per_launch": comp_b,
+         "launch_ms": round(t_comp, 4)}]
+
+    # ---- end to end through the host-buffer entry point
+    E = min(args.e2e_layers, L)
+    hc = api.HostCompressor(lay0.cu_seqlens.cpu(), Hq, Hkv, d, B, device=dev)
+    host = [tuple(t.cpu().pin_memory() for t in (l.Q, l.K, l.V)) for l in layers[:E]]
+    hc(*host[0], a, b, R)
+    torch.cuda.synchronize()
+    D.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.e2e_steps):
+        for hq in host:
+            hc(*hq, a, b, R)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = D.max(t0.elapsed_time(t1)) / args.e2e_steps
+    e2e = {"value": D.world * E * sum(lay0.lens) / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": hc.h2d_bytes * E, "d2h_bytes_per_step": hc.d2h_bytes * E,
+           "step": f"{E} layers through waits_compress_host (pinned host buffers)",
+           "ms_per_step": round(e2e_ms, 3)}
+
+    cpu = None
+    if D.rank == 0 and D.world == 1 and not args.no_cpu_baseline:
+        dt, threads = cpu_oracle_sample(lay0, a, b, R, B)
+        cpu = {"value": sum(lay0.lens) / (dt * Hkv), "unit": UNIT, "cores": threads,
+               "kind": "oracle",
+               "sample": f"fp64 numpy oracle on KV head 0 of layer 0 (its {Hq // Hkv} query "
+                         f"heads: score+select+compact), {dt:.2f} s, scaled x{Hkv} to a "
+                         f"whole layer"}
+
+    if D.rank == 0:
+        out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": D.world, "steps": K,
+               "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+               "config": config_dict(args, L, lay0.lens, wl.CONFIGS[CONFIG]),
+               "roofline": roof, "roofline_other": other, "cpu_baseline": cpu, "e2e": e2e,
+               "gpu_launches": KERNELS_PER_LAYER * L * K, "clocks": clk,
+               "per_layer_us": {"score": round(t_score * 1e3, 2),
+                                "select": round(t_sel * 1e3, 2),
+                                "compact": round(t_comp * 1e3, 2)},
+               "active_logits_per_layer": logits}
+        print(json.dumps(out), flush=True)
+    D.close()
+
+
+# ------------------------------------------------------------- reference ---
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    spec = wl.CONFIGS[CONFIG]
+    a, b = spec.actions[0]
+    R, B, L = spec.recent, args.budget, args.layers
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    lay = wl.make_layer(CONFIG, layer=0, device=dev)
+    Hkv = lay.K.shape[1]
+    times, threads = [], 1
+    for k in range(args.warmup + args.steps):
+        dt, threads = cpu_oracle_sample(lay, a, b, R, B, g=k % Hkv)
+        if k >= args.warmup:
+            times.append(dt)
+    per_layer = statistics.mean(times) * Hkv
+    value = sum(lay.lens) / per_layer
+    sample = (f"each step: the fp64 numpy oracle on one KV head of layer 0 "
+              f"(score+select+compact), scaled x{Hkv} to a whole layer")
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": per_layer * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": config_dict(args, L, lay.lens, spec),
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,199 @@
+/*
+ * waits.h -- C ABI of libwaits.so, the B200 (sm_100a) WAITS prefill
+ * KV-eviction path: score -> select -> compact.
+ *
+ * Method source: the WAITS README (stig.sh/Dirac-Notation/A2SF).
+ *   - Opening summary: keys are retained by an accumulative attention score
+ *     whose query rows are weighted by the sigmoid forgetting curve
+ *     w[q] = 1 / (1 + exp(-a * (q - (N - b - 0.5)))).
+ *   - Quickstart: init_cache keys "sigmoid_a" (a), "recent_budget" (R) and
+ *     "select_budget" (B); Evaluation: the window b is the --window flag.
+ *
+ * Conventions shared by every entry point
+ *   Layout    Packed varlen ("THD"): Q is [T, Hq, d], K and V are [T, Hkv, d],
+ *             bf16, row-major, d contiguous; sequence i owns tokens
+ *             [cu_seqlens[i], cu_seqlens[i+1]).  T = total_tokens.  Query
+ *             head h reads KV head h / G with G = Hq / Hkv.
+ *   Positions Sequence-local and 0-based: q, k in [0, N_i).
+ *   Memory    Every pointer is DEVICE memory owned by the caller unless its
+ *             comment says HOST.  The library allocates nothing and keeps no
+ *             state between calls; scratch lives in the caller's workspace.
+ *             Q, K, V must be 16-byte aligned.
+ *   Streams   `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *             default stream).  Calls only enqueue work on it and return; the
+ *             outputs are valid once the stream reaches that point.
+ *   Errors    Arguments are validated on the host before anything is
+ *             enqueued; a non-OK status means nothing was launched.  Problems
+ *             only the device can see (malformed cu_seqlens, an index out of
+ *             range handed to waits_compact, a bounded wait that gave up) set
+ *             bits of a status word in the workspace and the affected work is
+ *             skipped, never performed out of bounds; read it with
+ *             waits_read_device_status().
+ *   Inputs    Q and K must be finite (non-finite values give unspecified
+ *             scores but never out-of-bounds accesses).
+ */
+#ifndef WAITS_H
+#define WAITS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WAITS_ABI_VERSION 1
+
+typedef enum waits_status {
+  WAITS_OK = 0,
+  WAITS_ERR_ARG = 1,          /* null pointer, misalignment, bad a/b/R/B   */
+  WAITS_ERR_SHAPE = 2,        /* inconsistent or out-of-range shape        */
+  WAITS_ERR_UNSUPPORTED = 3,  /* head_dim not 64/128, G > 128, ...         */
+  WAITS_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than required   */
+  WAITS_ERR_CUDA = 5,         /* a CUDA runtime call failed                */
+  WAITS_ERR_TIMEOUT = 6,      /* device status: a bounded wait gave up     */
+  WAITS_ERR_DEVICE = 7        /* device status: other device-side problem  */
+} waits_status;
+
+/* Bits of the device status word (waits_read_device_status). */
+#define WAITS_DEV_TIMEOUT        0x1u  /* a bounded spin/mbarrier wait expired */
+#define WAITS_DEV_BAD_SEQLENS    0x2u  /* cu_seqlens not 0 <= ... <= T, or N > max_seqlen */
+#define WAITS_DEV_PLAN_OVERFLOW  0x4u  /* internal: plan larger than its bound */
+#define WAITS_DEV_BAD_INDEX      0x8u  /* waits_compact saw idx outside [0, N) */
+
+typedef struct waits_shape {
+  int32_t nseq;             /* sequences in the packed batch, >= 1             */
+  int32_t total_tokens;     /* T = cu_seqlens[nseq], >= 1                      */
+  int32_t max_seqlen;       /* upper bound on every N_i (host-side value)      */
+  int32_t num_q_heads;      /* Hq, a multiple of num_kv_heads                  */
+  int32_t num_kv_heads;     /* Hkv >= 1                                        */
+  int32_t head_dim;         /* d, 64 or 128                                    */
+  const int32_t* cu_seqlens;/* DEVICE, int32 [nseq + 1], cu[0] = 0, non-decreasing */
+} waits_shape;
+
+/* Library ABI version (WAITS_ABI_VERSION of the build). */
+int32_t waits_abi_version(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char* waits_strerror(waits_status status);
+
+/*
+ * Bytes of device workspace that waits_score / waits_compress need for
+ * `shape` (any a, b, R, B).  Host-only; touches no device state.
+ * Errors: WAITS_ERR_ARG if shape or bytes is NULL; shape errors as below.
+ */
+waits_status waits_workspace_size(const waits_shape* shape, size_t* bytes);
+
+/*
+ * Accumulative forgetting-curve score (README opening summary).  For every
+ * sequence, KV head g and key k:
+ *   scores[g * T + cu[i] + k] =
+ *     sum_{h in group g} sum_{q >= k} w[q] * softmax_k'(Q[q,h].K[k',g] / sqrt(d))[k]
+ * with w from the forgetting curve, N = N_i, and the sum restricted to rows
+ * whose fp32 weight 1.0f/(1.0f+expf(-a*(q-c))) is non-zero (the others add
+ * less than 1e-37 each).
+ *   Q, K       bf16 [T, Hq, d] / [T, Hkv, d]
+ *   a          slope, finite and >= 0 (0 gives H2O; 1e4 a step)
+ *   b          window, >= 0
+ *   scores     fp32 [Hkv, T], written for every token
+ *   workspace  >= waits_workspace_size() bytes, 256-byte aligned
+ * Errors: ARG (null, misaligned, a < 0 or non-finite, b < 0), SHAPE,
+ * UNSUPPORTED, WORKSPACE, CUDA.
+ */
+waits_status waits_score(const waits_shape* shape, const void* Q, const void* K,
+                         float a, int32_t b, float* scores, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * Selection (README Quickstart budgets).  Per sequence i and KV head g:
+ * keep the recent window [N-R, N) and the B-R positions of [0, N-R) with the
+ * largest score, ties to the lower index; N <= B keeps every position.
+ *   idx        int32 [nseq, Hkv, B]: kept positions, sequence-local,
+ *              ascending; entries j >= kept_len[i] are -1
+ *   kept_len   int32 [nseq]: min(N_i, B)
+ *   workspace  may be NULL (this call needs none); kept for ABI symmetry
+ * Errors: ARG (null, R < 0, R > B, B < 1), SHAPE, CUDA.
+ */
+waits_status waits_select(const waits_shape* shape, const float* scores,
+                          int32_t R, int32_t B, int32_t* idx, int32_t* kept_len,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Compaction ("retaining key-value pairs", README opening summary):
+ *   K_out[i, g, j, :] = K[cu[i] + idx[i, g, j], g, :] for j < kept_len[i],
+ *   zero for j >= kept_len[i]; same for V.  Bit-exact copy.
+ *   K_out, V_out  bf16 [nseq, Hkv, B, d], 16-byte aligned
+ * An idx entry outside [0, N_i) sets WAITS_DEV_BAD_INDEX (in `workspace` if
+ * given) and that row is written as zeros.
+ * Errors: ARG, SHAPE, UNSUPPORTED, CUDA.
+ */
+waits_status waits_compact(const waits_shape* shape, const void* K, const void* V,
+                           const int32_t* idx, const int32_t* kept_len, int32_t B,
+                           void* K_out, void* V_out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * score -> select -> compact in one call, all enqueued on `stream`.
+ * Arguments as above; `scores` is an output too.
+ */
+waits_status waits_compress(const waits_shape* shape, const void* Q, const void* K,
+                            const void* V, float a, int32_t b, int32_t R, int32_t B,
+                            float* scores, int32_t* idx, int32_t* kept_len,
+                            void* K_out, void* V_out, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* Device buffers that waits_compress_host stages through (caller-owned). */
+typedef struct waits_device_buffers {
+  void* Q;          /* bf16 [T, Hq, d]  */
+  void* K;          /* bf16 [T, Hkv, d] */
+  void* V;          /* bf16 [T, Hkv, d] */
+  float* scores;    /* fp32 [Hkv, T]    */
+  int32_t* idx;     /* [nseq, Hkv, B]   */
+  int32_t* kept_len;/* [nseq]           */
+  void* K_out;      /* bf16 [nseq, Hkv, B, d] */
+  void* V_out;      /* bf16 [nseq, Hkv, B, d] */
+  int32_t* cu_seqlens; /* [nseq + 1]    */
+} waits_device_buffers;
+
+/*
+ * Host-buffer variant of waits_compress: copies the inputs from HOST memory
+ * (pinned memory makes the copies asynchronous), runs the path, and copies
+ * idx, kept_len, K_out and V_out back to HOST memory, all on `stream`.
+ * Only the rows the scorer can read are sent: each sequence's query rows
+ * from a conservative lower bound of the first non-zero-weight row on, and
+ * all of K and V.  The call returns once the copies are enqueued; the host
+ * outputs are valid after the stream is synchronised.
+ *   cu_seqlens_host  HOST int32 [nseq + 1]
+ *   Q_host, K_host, V_host, idx_host, kept_len_host, K_out_host,
+ *   V_out_host       HOST, same layouts as the device versions
+ *   dev              device staging buffers; dev->cu_seqlens receives the
+ *                    offsets and shape->cu_seqlens is ignored
+ *   h2d_bytes, d2h_bytes  optional HOST out: bytes copied each way
+ * Errors: as waits_compress, plus SHAPE if cu_seqlens_host is inconsistent.
+ */
+waits_status waits_compress_host(const waits_shape* shape,
+                                 const int32_t* cu_seqlens_host,
+                                 const void* Q_host, const void* K_host,
+                                 const void* V_host, float a, int32_t b,
+                                 int32_t R, int32_t B, int32_t* idx_host,
+                                 int32_t* kept_len_host, void* K_out_host,
+                                 void* V_out_host,
+                                 const waits_device_buffers* dev,
+                                 void* workspace, size_t workspace_bytes,
+                                 void* stream, size_t* h2d_bytes,
+                                 size_t* d2h_bytes);
+
+/*
+ * Synchronise `stream` and read the device status word of `workspace`
+ * (bits WAITS_DEV_*; 0 = clean).  The word is cleared at the start of every
+ * waits_score / waits_compress.  Errors: ARG, WORKSPACE, CUDA.
+ */
+waits_status waits_read_device_status(const void* workspace,
+                                      size_t workspace_bytes, void* stream,
+                                      uint32_t* status_bits);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WAITS_H */

@@ -1,0 +1,237 @@
+"""Python binding of libwaits.so: argument marshalling for torch tensors.
+
+Every step of the path runs in the library's CUDA kernels; this module only
+checks tensor shapes/dtypes, allocates outputs with torch, and passes raw
+pointers and the current CUDA stream.  Names follow the WAITS README
+Quickstart (``sigmoid_a``, ``recent_budget``, ``select_budget``/``budget``)
+and Evaluation (``window`` = b).
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(name, t, dtype):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def make_shape(cu_seqlens: torch.Tensor, total_tokens: int, max_seqlen: int,
+               num_q_heads: int, num_kv_heads: int, head_dim: int) -> _lib.Shape:
+    return _lib.Shape(int(cu_seqlens.numel() - 1), int(total_tokens),
+                      int(max_seqlen), int(num_q_heads), int(num_kv_heads),
+                      int(head_dim), cu_seqlens.data_ptr())
+
+
+def workspace_bytes(shape: _lib.Shape) -> int:
+    lib = _lib.load()
+    n = ctypes.c_size_t(0)
+    _lib.check("waits_workspace_size", lib.waits_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return int(n.value)
+
+
+def _max_seqlen(cu_seqlens, max_seqlen):
+    if max_seqlen is not None:
+        return int(max_seqlen)
+    cu = cu_seqlens.to("cpu")
+    return int((cu[1:] - cu[:-1]).max()) if cu.numel() > 1 else 0
+
+
+class Compressor:
+    """Reusable workspace + outputs for one packed-batch shape.
+
+    ``Compressor(cu_seqlens, T, max_seqlen, Hq, Hkv, d, budget)`` allocates
+    the workspace and the output tensors once; each call enqueues
+    score -> select -> compact on the current stream.
+    """
+
+    def __init__(self, cu_seqlens: torch.Tensor, total_tokens: int,
+                 max_seqlen: int, num_q_heads: int, num_kv_heads: int,
+                 head_dim: int, budget: int):
+        _need_cuda("cu_seqlens", cu_seqlens, torch.int32)
+        self.lib = _lib.load()
+        self.cu = cu_seqlens
+        self.dev = cu_seqlens.device
+        self.shape = make_shape(cu_seqlens, total_tokens, max_seqlen,
+                                num_q_heads, num_kv_heads, head_dim)
+        self.nseq = cu_seqlens.numel() - 1
+        self.T, self.Hq, self.Hkv, self.d = total_tokens, num_q_heads, num_kv_heads, head_dim
+        self.B = int(budget)
+        self.ws_bytes = workspace_bytes(self.shape)
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.dev)
+        self.scores = torch.empty((num_kv_heads, total_tokens), dtype=torch.float32, device=self.dev)
+        self.idx = torch.empty((self.nseq, num_kv_heads, self.B), dtype=torch.int32, device=self.dev)
+        self.kept_len = torch.empty((self.nseq,), dtype=torch.int32, device=self.dev)
+        self.K_out = torch.empty((self.nseq, num_kv_heads, self.B, head_dim), dtype=torch.bfloat16, device=self.dev)
+        self.V_out = torch.empty_like(self.K_out)
+
+    def check_inputs(self, Q, K, V=None):
+        _need_cuda("Q", Q, torch.bfloat16)
+        _need_cuda("K", K, torch.bfloat16)
+        if tuple(Q.shape) != (self.T, self.Hq, self.d) or tuple(K.shape) != (self.T, self.Hkv, self.d):
+            raise ValueError("Q/K shapes do not match the compressor's shape")
+        if V is not None:
+            _need_cuda("V", V, torch.bfloat16)
+            if V.shape != K.shape:
+                raise ValueError("V must have K's shape")
+
+    def __call__(self, Q, K, V, sigmoid_a: float, window: int, recent_budget: int):
+        self.check_inputs(Q, K, V)
+        st = self.lib.waits_compress(
+            ctypes.byref(self.shape), _ptr(Q), _ptr(K), _ptr(V), float(sigmoid_a),
+            int(window), int(recent_budget), self.B, _ptr(self.scores), _ptr(self.idx),
+            _ptr(self.kept_len), _ptr(self.K_out), _ptr(self.V_out), _ptr(self.workspace),
+            self.ws_bytes, _stream(self.dev))
+        _lib.check("waits_compress", st)
+        return self.K_out, self.V_out, self.idx, self.kept_len, self.scores
+
+    def score(self, Q, K, sigmoid_a: float, window: int):
+        self.check_inputs(Q, K)
+        st = self.lib.waits_score(ctypes.byref(self.shape), _ptr(Q), _ptr(K), float(sigmoid_a),
+                                  int(window), _ptr(self.scores), _ptr(self.workspace),
+                                  self.ws_bytes, _stream(self.dev))
+        _lib.check("waits_score", st)
+        return self.scores
+
+    def device_status(self) -> int:
+        v = ctypes.c_uint32(0)
+        _lib.check("waits_read_device_status", self.lib.waits_read_device_status(
+            _ptr(self.workspace), self.ws_bytes, _stream(self.dev), ctypes.byref(v)))
+        return int(v.value)
+
+
+def score(Q: torch.Tensor, K: torch.Tensor, cu_seqlens: torch.Tensor, *,
+          sigmoid_a: float, window: int, max_seqlen: Optional[int] = None) -> torch.Tensor:
+    """fp32 scores ``[Hkv, T]`` (``waits_score``)."""
+    T, Hq, d = Q.shape
+    c = Compressor(cu_seqlens, T, _max_seqlen(cu_seqlens, max_seqlen), Hq, K.shape[1], d, 1)
+    return c.score(Q, K, sigmoid_a, window)
+
+
+def select(scores: torch.Tensor, cu_seqlens: torch.Tensor, *, recent_budget: int,
+           budget: int, max_seqlen: Optional[int] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """``(idx [nseq, Hkv, B] int32, kept_len [nseq] int32)`` (``waits_select``)."""
+    _need_cuda("scores", scores, torch.float32)
+    _need_cuda("cu_seqlens", cu_seqlens, torch.int32)
+    lib = _lib.load()
+    Hkv, T = scores.shape
+    nseq = cu_seqlens.numel() - 1
+    shape = make_shape(cu_seqlens, T, _max_seqlen(cu_seqlens, max_seqlen), Hkv, Hkv, 64)
+    idx = torch.empty((nseq, Hkv, int(budget)), dtype=torch.int32, device=scores.device)
+    kept = torch.empty((nseq,), dtype=torch.int32, device=scores.device)
+    st = lib.waits_select(ctypes.byref(shape), _ptr(scores), int(recent_budget), int(budget),
+                          _ptr(idx), _ptr(kept), None, 0, _stream(scores.device))
+    _lib.check("waits_select", st)
+    return idx, kept
+
+
+def compact(K: torch.Tensor, V: torch.Tensor, cu_seqlens: torch.Tensor, idx: torch.Tensor,
+            kept_len: torch.Tensor, *, max_seqlen: Optional[int] = None,
+            workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """``(K_out, V_out)`` bf16 ``[nseq, Hkv, B, d]`` (``waits_compact``)."""
+    _need_cuda("K", K, torch.bfloat16)
+    _need_cuda("V", V, torch.bfloat16)
+    _need_cuda("idx", idx, torch.int32)
+    _need_cuda("kept_len", kept_len, torch.int32)
+    lib = _lib.load()
+    T, Hkv, d = K.shape
+    nseq, _, B = idx.shape
+    shape = make_shape(cu_seqlens, T, _max_seqlen(cu_seqlens, max_seqlen), Hkv, Hkv, d)
+    Ko = torch.empty((nseq, Hkv, B, d), dtype=torch.bfloat16, device=K.device)
+    Vo = torch.empty_like(Ko)
+    ws_b = 0 if workspace is None else workspace.numel()
+    st = lib.waits_compact(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(idx), _ptr(kept_len),
+                           int(B), _ptr(Ko), _ptr(Vo), _ptr(workspace), ws_b,
+                           _stream(K.device))
+    _lib.check("waits_compact", st)
+    return Ko, Vo
+
+
+def compress(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, *,
+             sigmoid_a: float, window: int, recent_budget: int, budget: int,
+             max_seqlen: Optional[int] = None):
+    """WAITS prefill compression of one layer (``waits_compress``).
+
+    Returns ``(K_out, V_out, idx, kept_len, scores)``.
+    """
+    T, Hq, d = q.shape
+    c = Compressor(cu_seqlens, T, _max_seqlen(cu_seqlens, max_seqlen), Hq, k.shape[1], d,
+                   budget)
+    return c(q, k, v, sigmoid_a, window, recent_budget)
+
+
+class HostCompressor:
+    """``waits_compress_host``: inputs and outputs in (pinned) host memory,
+    device staging buffers owned here."""
+
+    def __init__(self, cu_seqlens_host: torch.Tensor, num_q_heads: int, num_kv_heads: int,
+                 head_dim: int, budget: int, device="cuda"):
+        self.lib = _lib.load()
+        cu = cu_seqlens_host.to(torch.int32).contiguous()
+        self.cu_host = cu.pin_memory() if not cu.is_pinned() else cu
+        self.nseq = cu.numel() - 1
+        self.T = int(cu[-1])
+        self.max_seqlen = int((cu[1:] - cu[:-1]).max())
+        self.B = int(budget)
+        self.Hq, self.Hkv, self.d = num_q_heads, num_kv_heads, head_dim
+        dev = torch.device(device)
+        self.dev = dev
+        bf = torch.bfloat16
+        self.dQ = torch.zeros((self.T, num_q_heads, head_dim), dtype=bf, device=dev)
+        self.dK = torch.empty((self.T, num_kv_heads, head_dim), dtype=bf, device=dev)
+        self.dV = torch.empty_like(self.dK)
+        self.dcu = torch.empty((self.nseq + 1,), dtype=torch.int32, device=dev)
+        self.dscores = torch.empty((num_kv_heads, self.T), dtype=torch.float32, device=dev)
+        self.didx = torch.empty((self.nseq, num_kv_heads, self.B), dtype=torch.int32, device=dev)
+        self.dkept = torch.empty((self.nseq,), dtype=torch.int32, device=dev)
+        self.dKo = torch.empty((self.nseq, num_kv_heads, self.B, head_dim), dtype=bf, device=dev)
+        self.dVo = torch.empty_like(self.dKo)
+        self.shape = make_shape(self.dcu, self.T, self.max_seqlen, num_q_heads, num_kv_heads,
+                                head_dim)
+        self.ws_bytes = workspace_bytes(self.shape)
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.bufs = _lib.DeviceBuffers(
+            self.dQ.data_ptr(), self.dK.data_ptr(), self.dV.data_ptr(), self.dscores.data_ptr(),
+            self.didx.data_ptr(), self.dkept.data_ptr(), self.dKo.data_ptr(),
+            self.dVo.data_ptr(), self.dcu.data_ptr())
+        pin = dict(pin_memory=True)
+        self.idx = torch.empty((self.nseq, num_kv_heads, self.B), dtype=torch.int32, **pin)
+        self.kept_len = torch.empty((self.nseq,), dtype=torch.int32, **pin)
+        self.K_out = torch.empty((self.nseq, num_kv_heads, self.B, head_dim), dtype=bf, **pin)
+        self.V_out = torch.empty_like(self.K_out).pin_memory()
+        self.h2d_bytes = 0
+        self.d2h_bytes = 0
+
+    def __call__(self, Q_host, K_host, V_host, sigmoid_a: float, window: int,
+                 recent_budget: int):
+        for n, t in (("Q", Q_host), ("K", K_host), ("V", V_host)):
+            if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+                raise ValueError(f"{n} must be a contiguous bf16 host tensor")
+        up, down = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        st = self.lib.waits_compress_host(
+            ctypes.byref(self.shape), _ptr(self.cu_host), _ptr(Q_host), _ptr(K_host),
+            _ptr(V_host), float(sigmoid_a), int(window), int(recent_budget), self.B,
+            _ptr(self.idx), _ptr(self.kept_len), _ptr(self.K_out), _ptr(self.V_out),
+            ctypes.byref(self.bufs), _ptr(self.workspace), self.ws_bytes, _stream(self.dev),
+            ctypes.byref(up), ctypes.byref(down))
+        _lib.check("waits_compress_host", st)
+        self.h2d_bytes, self.d2h_bytes = int(up.value), int(down.value)
+        return self.K_out, self.V_out, self.idx, self.kept_len

@@ -1,0 +1,77 @@
+// Walking the work plan: which steps (streamed tiles) of which entries a
+// persistent CTA owns, and the per-tile geometry both scorer passes share.
+#pragma once
+
+#include "waits_internal.cuh"
+
+namespace waits {
+
+// CTA `cta` of `P` owns global steps [ceil(cta*S/P), ceil((cta+1)*S/P)); a
+// maximal run of them inside one entry is a unit.
+struct UnitIter {
+  const Entry* E;
+  int nE;
+  int64_t hi;     // end of this CTA's step range
+  int e;          // current entry
+  int64_t pos;    // next global step
+  int cta;
+
+  __device__ bool init(const Entry* E_, int nE_, int64_t S, int P, int cta_) {
+    E = E_; nE = nE_; cta = cta_;
+    if (cta >= P || nE <= 0 || S <= 0) return false;
+    const int64_t lo = ((int64_t)cta * S + P - 1) / P;
+    hi = ((int64_t)(cta + 1) * S + P - 1) / P;
+    if (lo >= hi) return false;
+    int a = 0, b = nE - 1;
+    while (a < b) {
+      const int m = (a + b + 1) / 2;
+      if (E[m].sbase <= lo) a = m; else b = m - 1;
+    }
+    e = a;
+    pos = lo;
+    return true;
+  }
+  // Next unit: entry index, local step range [st0, st1) and unit slot.
+  __device__ bool next(int& ei, int& st0, int& st1, int& unit) {
+    if (pos >= hi || e >= nE) return false;
+    const Entry& en = E[e];
+    const int64_t end = en.sbase + en.n_steps;
+    const int64_t stop = end < hi ? end : hi;
+    ei = e;
+    st0 = (int)(pos - en.sbase);
+    st1 = (int)(stop - en.sbase);
+    unit = en.unit_base + (cta - en.first_cta);
+    pos = stop;
+    if (stop == end) ++e;
+    return true;
+  }
+};
+
+// Geometry of Q tile j of a sequence (packed rows r = token * G + head).
+__device__ inline int qtile_first_tok(const SeqInfo& si, int j, int tokq) {
+  return si.q0 + j * tokq;
+}
+__device__ inline int qtile_last_tok(const SeqInfo& si, int j, int tokq) {
+  const int e = si.q0 + (j + 1) * tokq;
+  return (e < si.len ? e : si.len) - 1;
+}
+// Some row of Q tile j sees some key of K tile kt (causal).
+__device__ inline bool pair_live(const SeqInfo& si, int j, int kt, int tokq) {
+  return qtile_last_tok(si, j, tokq) >= kt * kTile;
+}
+// Every row of Q tile j sees every key of K tile kt.
+__device__ inline bool pair_full(const SeqInfo& si, int j, int kt, int tokq) {
+  return qtile_first_tok(si, j, tokq) >= kt * kTile + kTile - 1;
+}
+
+__device__ inline float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Largest partial sum kept before the reference maximum of a row is moved
+// up (2^64: far from fp32 overflow even after adding a whole tile).
+constexpr float kRebaseLimit = 1.8446744073709552e19f;
+
+}  // namespace waits

@@ -1,0 +1,320 @@
+// C ABI of libwaits.so: host-side validation, workspace carving and launches
+// on the caller's stream.  Declarations and contracts: include/waits.h.
+#include <cmath>
+#include <cstring>
+
+#include "waits_internal.cuh"
+
+using namespace waits;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+waits_status check_shape(const waits_shape* s) {
+  if (!s || !s->cu_seqlens) return WAITS_ERR_ARG;
+  if (s->nseq < 1 || s->total_tokens < 1 || s->max_seqlen < 1 || s->num_kv_heads < 1 ||
+      s->num_q_heads < 1)
+    return WAITS_ERR_SHAPE;
+  if (s->num_q_heads % s->num_kv_heads) return WAITS_ERR_SHAPE;
+  if (s->max_seqlen > s->total_tokens) return WAITS_ERR_SHAPE;
+  if (s->head_dim != 64 && s->head_dim != 128) return WAITS_ERR_UNSUPPORTED;
+  if (s->num_q_heads / s->num_kv_heads > kTile) return WAITS_ERR_UNSUPPORTED;
+  // every flat index below fits comfortably in 64 bits; keep T*Hq*d in 2^40
+  const double elems = (double)s->total_tokens * s->num_q_heads * s->head_dim;
+  if (elems > 1099511627776.0 || s->nseq > s->total_tokens) return WAITS_ERR_SHAPE;
+  return WAITS_OK;
+}
+
+Layout layout_of(const waits_shape* s) {
+  return make_layout(s->nseq, s->total_tokens, s->num_q_heads, s->num_kv_heads);
+}
+
+waits_status check_ws(const waits_shape* s, const void* ws, size_t bytes) {
+  if (!ws) return WAITS_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return WAITS_ERR_ARG;
+  if (bytes < layout_of(s).total) return WAITS_ERR_WORKSPACE;
+  return WAITS_OK;
+}
+
+waits_status check_budget(int32_t R, int32_t B) {
+  if (B < 1 || R < 0 || R > B) return WAITS_ERR_ARG;
+  return WAITS_OK;
+}
+
+int grid_size() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms < kMaxGrid ? sms : kMaxGrid;
+}
+
+uint32_t* status_word(void* ws, size_t bytes) {
+  if (!ws || bytes < sizeof(PlanHeader) || !aligned(ws, 256)) return nullptr;
+  return &reinterpret_cast<PlanHeader*>(ws)->status;
+}
+
+waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, float a,
+                           int32_t b, float* scores, void* ws, cudaStream_t st) {
+  const Layout L = layout_of(s);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const int grid = grid_size();
+  if (grid <= 0) return WAITS_ERR_CUDA;
+  PlanArgs pa{};
+  pa.cu = s->cu_seqlens;
+  pa.nseq = s->nseq;
+  pa.T = s->total_tokens;
+  pa.max_seqlen = s->max_seqlen;
+  pa.Hq = s->num_q_heads;
+  pa.Hkv = s->num_kv_heads;
+  pa.G = s->num_q_heads / s->num_kv_heads;
+  pa.tokq = tokens_per_qtile(pa.G);
+  pa.a = a;
+  pa.b = b;
+  pa.grid = grid;
+  pa.hdr = reinterpret_cast<PlanHeader*>(base + L.header);
+  pa.seqs = reinterpret_cast<SeqInfo*>(base + L.seqs);
+  pa.e1 = reinterpret_cast<Entry*>(base + L.e1);
+  pa.e2 = reinterpret_cast<Entry*>(base + L.e2);
+  pa.c1 = reinterpret_cast<uint32_t*>(base + L.c1);
+  pa.c2 = reinterpret_cast<uint32_t*>(base + L.c2);
+  pa.max_e1 = L.max_e1;
+  pa.max_e2 = L.max_e2;
+  pa.max_u1 = L.max_u1;
+  pa.max_u2 = L.max_u2;
+  pa.scores = scores;
+  if (launch_plan(pa, st) != cudaSuccess) return WAITS_ERR_CUDA;
+
+  PassArgs p{};
+  p.Q = static_cast<const uint16_t*>(Q);
+  p.K = static_cast<const uint16_t*>(K);
+  p.T = s->total_tokens;
+  p.Hq = s->num_q_heads;
+  p.Hkv = s->num_kv_heads;
+  p.G = pa.G;
+  p.tokq = pa.tokq;
+  p.d = s->head_dim;
+  p.a = a;
+  p.b = b;
+  p.scale2 = (float)(1.4426950408889634 / std::sqrt((double)s->head_dim));
+  p.hdr = pa.hdr;
+  p.seqs = pa.seqs;
+  p.e1 = pa.e1;
+  p.e2 = pa.e2;
+  p.c1 = pa.c1;
+  p.c2 = pa.c2;
+  p.bias = reinterpret_cast<float*>(base + L.bias);
+  p.part1 = reinterpret_cast<float2*>(base + L.part1);
+  p.part2 = reinterpret_cast<float*>(base + L.part2);
+  p.scores = scores;
+  p.status = &pa.hdr->status;
+  if (launch_score_passes(p, grid, st) != cudaSuccess) return WAITS_ERR_CUDA;
+  return WAITS_OK;
+}
+
+waits_status check_score_args(const waits_shape* s, const void* Q, const void* K, float a,
+                              int32_t b, const float* scores) {
+  if (!Q || !K || !scores) return WAITS_ERR_ARG;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(scores, 4)) return WAITS_ERR_ARG;
+  if (!std::isfinite(a) || a < 0.0f || b < 0) return WAITS_ERR_ARG;
+  (void)s;
+  return WAITS_OK;
+}
+
+waits_status check_select_args(const float* scores, int32_t R, int32_t B, const int32_t* idx,
+                               const int32_t* kept_len) {
+  if (!scores || !idx || !kept_len) return WAITS_ERR_ARG;
+  return check_budget(R, B);
+}
+
+waits_status check_compact_args(const void* K, const void* V, const int32_t* idx,
+                                const int32_t* kept_len, int32_t B, const void* Ko,
+                                const void* Vo) {
+  if (!K || !V || !idx || !kept_len || !Ko || !Vo) return WAITS_ERR_ARG;
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(Ko, 16) || !aligned(Vo, 16))
+    return WAITS_ERR_ARG;
+  if (B < 1) return WAITS_ERR_ARG;
+  return WAITS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t waits_abi_version(void) { return WAITS_ABI_VERSION; }
+
+const char* waits_strerror(waits_status st) {
+  switch (st) {
+    case WAITS_OK: return "ok";
+    case WAITS_ERR_ARG: return "invalid argument (null, misaligned, or a/b/R/B out of range)";
+    case WAITS_ERR_SHAPE: return "invalid or inconsistent shape";
+    case WAITS_ERR_UNSUPPORTED: return "unsupported configuration (head_dim must be 64 or 128, G <= 128)";
+    case WAITS_ERR_WORKSPACE: return "workspace missing or smaller than waits_workspace_size()";
+    case WAITS_ERR_CUDA: return "a CUDA runtime call failed";
+    case WAITS_ERR_TIMEOUT: return "a bounded device-side wait expired";
+    case WAITS_ERR_DEVICE: return "device-side error (see WAITS_DEV_* status bits)";
+  }
+  return "unknown status";
+}
+
+waits_status waits_workspace_size(const waits_shape* shape, size_t* bytes) {
+  if (!bytes) return WAITS_ERR_ARG;
+  const waits_status st = check_shape(shape);
+  if (st != WAITS_OK) return st;
+  *bytes = layout_of(shape).total;
+  return WAITS_OK;
+}
+
+waits_status waits_score(const waits_shape* shape, const void* Q, const void* K, float a,
+                         int32_t b, float* scores, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  waits_status st = check_shape(shape);
+  if (st == WAITS_OK) st = check_score_args(shape, Q, K, a, b, scores);
+  if (st == WAITS_OK) st = check_ws(shape, workspace, workspace_bytes);
+  if (st != WAITS_OK) return st;
+  return enqueue_score(shape, Q, K, a, b, scores, workspace, static_cast<cudaStream_t>(stream));
+}
+
+waits_status waits_select(const waits_shape* shape, const float* scores, int32_t R, int32_t B,
+                          int32_t* idx, int32_t* kept_len, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  waits_status st = check_shape(shape);
+  if (st == WAITS_OK) st = check_select_args(scores, R, B, idx, kept_len);
+  if (st != WAITS_OK) return st;
+  if (launch_select(scores, shape->cu_seqlens, shape->nseq, shape->total_tokens,
+                    shape->num_kv_heads, R, B, idx, kept_len,
+                    status_word(workspace, workspace_bytes),
+                    static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return WAITS_ERR_CUDA;
+  return WAITS_OK;
+}
+
+waits_status waits_compact(const waits_shape* shape, const void* K, const void* V,
+                           const int32_t* idx, const int32_t* kept_len, int32_t B, void* K_out,
+                           void* V_out, void* workspace, size_t workspace_bytes, void* stream) {
+  waits_status st = check_shape(shape);
+  if (st == WAITS_OK) st = check_compact_args(K, V, idx, kept_len, B, K_out, V_out);
+  if (st != WAITS_OK) return st;
+  if (launch_compact(static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
+                     shape->cu_seqlens, idx, kept_len, shape->nseq, shape->num_kv_heads,
+                     shape->head_dim, B, static_cast<uint16_t*>(K_out),
+                     static_cast<uint16_t*>(V_out), status_word(workspace, workspace_bytes),
+                     static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return WAITS_ERR_CUDA;
+  return WAITS_OK;
+}
+
+waits_status waits_compress(const waits_shape* shape, const void* Q, const void* K,
+                            const void* V, float a, int32_t b, int32_t R, int32_t B,
+                            float* scores, int32_t* idx, int32_t* kept_len, void* K_out,
+                            void* V_out, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  waits_status st = check_shape(shape);
+  if (st == WAITS_OK) st = check_score_args(shape, Q, K, a, b, scores);
+  if (st == WAITS_OK) st = check_select_args(scores, R, B, idx, kept_len);
+  if (st == WAITS_OK) st = check_compact_args(K, V, idx, kept_len, B, K_out, V_out);
+  if (st == WAITS_OK) st = check_ws(shape, workspace, workspace_bytes);
+  if (st != WAITS_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = enqueue_score(shape, Q, K, a, b, scores, workspace, s);
+  if (st != WAITS_OK) return st;
+  uint32_t* status = status_word(workspace, workspace_bytes);
+  if (launch_select(scores, shape->cu_seqlens, shape->nseq, shape->total_tokens,
+                    shape->num_kv_heads, R, B, idx, kept_len, status, s) != cudaSuccess)
+    return WAITS_ERR_CUDA;
+  if (launch_compact(static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
+                     shape->cu_seqlens, idx, kept_len, shape->nseq, shape->num_kv_heads,
+                     shape->head_dim, B, static_cast<uint16_t*>(K_out),
+                     static_cast<uint16_t*>(V_out), status, s) != cudaSuccess)
+    return WAITS_ERR_CUDA;
+  return WAITS_OK;
+}
+
+waits_status waits_compress_host(const waits_shape* shape, const int32_t* cu_host,
+                                 const void* Q_host, const void* K_host, const void* V_host,
+                                 float a, int32_t b, int32_t R, int32_t B, int32_t* idx_host,
+                                 int32_t* kept_len_host, void* K_out_host, void* V_out_host,
+                                 const waits_device_buffers* dev, void* workspace,
+                                 size_t workspace_bytes, void* stream, size_t* h2d_bytes,
+                                 size_t* d2h_bytes) {
+  if (!shape || !cu_host || !dev || !Q_host || !K_host || !V_host || !idx_host ||
+      !kept_len_host || !K_out_host || !V_out_host || !dev->cu_seqlens)
+    return WAITS_ERR_ARG;
+  waits_shape sh = *shape;
+  sh.cu_seqlens = dev->cu_seqlens;
+  waits_status st = check_shape(&sh);
+  if (st != WAITS_OK) return st;
+  // host copy of the offsets: validate before sending anything
+  if (cu_host[0] != 0 || cu_host[sh.nseq] != sh.total_tokens) return WAITS_ERR_SHAPE;
+  for (int i = 0; i < sh.nseq; ++i) {
+    const int n = cu_host[i + 1] - cu_host[i];
+    if (n < 0 || n > sh.max_seqlen) return WAITS_ERR_SHAPE;
+  }
+  st = check_score_args(&sh, dev->Q, dev->K, a, b, dev->scores);
+  if (st == WAITS_OK) st = check_select_args(dev->scores, R, B, dev->idx, dev->kept_len);
+  if (st == WAITS_OK)
+    st = check_compact_args(dev->K, dev->V, dev->idx, dev->kept_len, B, dev->K_out, dev->V_out);
+  if (st == WAITS_OK) st = check_ws(&sh, workspace, workspace_bytes);
+  if (st != WAITS_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t qrow = (size_t)sh.num_q_heads * sh.head_dim * 2;
+  const size_t krow = (size_t)sh.num_kv_heads * sh.head_dim * 2;
+  size_t up = 0, down = 0;
+  auto h2d = [&](void* dst, const void* src, size_t n) {
+    up += n;
+    return cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, s) == cudaSuccess;
+  };
+  auto d2h = [&](void* dst, const void* src, size_t n) {
+    down += n;
+    return cudaMemcpyAsync(dst, src, n, cudaMemcpyDeviceToHost, s) == cudaSuccess;
+  };
+  bool ok = h2d(dev->cu_seqlens, cu_host, sizeof(int32_t) * (sh.nseq + 1));
+  // Query rows below this bound have -a*(q-c) > 88.73, so their fp32 weight
+  // is exactly 0 and the scorer never reads them.
+  for (int i = 0; i < sh.nseq && ok; ++i) {
+    const int lo = cu_host[i], N = cu_host[i + 1] - lo;
+    long long q_lo = 0;
+    if (a > 0.0f) {
+      const double c = (double)N - (double)b - 0.5;
+      q_lo = (long long)std::floor(c - 90.0 / (double)a) - 2;
+      if (q_lo < 0) q_lo = 0;
+      if (q_lo > N) q_lo = N;
+    }
+    const size_t off = (size_t)(lo + q_lo) * qrow;
+    if (N > q_lo) ok = h2d(static_cast<uint8_t*>(dev->Q) + off,
+                           static_cast<const uint8_t*>(Q_host) + off, (size_t)(N - q_lo) * qrow);
+  }
+  ok = ok && h2d(dev->K, K_host, (size_t)sh.total_tokens * krow);
+  ok = ok && h2d(dev->V, V_host, (size_t)sh.total_tokens * krow);
+  if (!ok) return WAITS_ERR_CUDA;
+  st = waits_compress(&sh, dev->Q, dev->K, dev->V, a, b, R, B, dev->scores, dev->idx,
+                      dev->kept_len, dev->K_out, dev->V_out, workspace, workspace_bytes, stream);
+  if (st != WAITS_OK) return st;
+  const size_t nidx = (size_t)sh.nseq * sh.num_kv_heads * B;
+  const size_t nout = nidx * sh.head_dim * 2;
+  ok = d2h(idx_host, dev->idx, nidx * sizeof(int32_t)) &&
+       d2h(kept_len_host, dev->kept_len, sh.nseq * sizeof(int32_t)) &&
+       d2h(K_out_host, dev->K_out, nout) && d2h(V_out_host, dev->V_out, nout);
+  if (!ok) return WAITS_ERR_CUDA;
+  if (h2d_bytes) *h2d_bytes = up;
+  if (d2h_bytes) *d2h_bytes = down;
+  return WAITS_OK;
+}
+
+waits_status waits_read_device_status(const void* workspace, size_t workspace_bytes,
+                                      void* stream, uint32_t* status_bits) {
+  if (!status_bits) return WAITS_ERR_ARG;
+  if (!workspace || workspace_bytes < sizeof(PlanHeader)) return WAITS_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return WAITS_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, &reinterpret_cast<const PlanHeader*>(workspace)->status,
+                      sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return WAITS_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return WAITS_ERR_CUDA;
+  *status_bits = v;
+  return WAITS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,201 @@
+// Internal definitions shared by the libwaits translation units: the
+// workspace layout, the work plan written by the planner kernel, the fp32
+// forgetting-curve weight, and small block-level helpers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "waits.h"
+
+namespace waits {
+
+// ---------------------------------------------------------------- tiling ---
+constexpr int kTile = 128;      // keys per K tile; max packed rows per Q tile
+constexpr int kMaxStat = 4;     // stationary tiles held by one work unit
+constexpr int kMaxGrid = 1024;  // upper bound on persistent CTAs (sizing)
+constexpr int kPlanThreads = 1024;
+
+// A Q tile packs `tokq` consecutive query positions x G heads of one KV
+// group: packed row r <-> position q0 + j*tokq + r / G, head g*G + r % G.
+__host__ __device__ inline int tokens_per_qtile(int G) { return kTile / G; }
+
+// ----------------------------------------------------------- plan types ---
+enum EntryMode : int32_t {
+  kModeP1 = 0,   // pass 1: stationary Q tiles, streamed K tiles
+  kModeP2Q = 1,  // pass 2: stationary Q tiles (all active rows), streamed K
+  kModeP2K = 2,  // pass 2: stationary K tiles, streamed Q tiles
+};
+
+struct SeqInfo {
+  int32_t start;   // cu_seqlens[s]
+  int32_t len;     // N
+  int32_t q0;      // first row with non-zero fp32 weight (len if none)
+  int32_t nqt;     // Q tiles covering rows [q0, N)
+  int32_t nkt;     // K tiles covering keys [0, N)
+  int32_t e1;      // first pass-1 entry of this sequence
+  int32_t e2;      // first pass-2 entry of this sequence
+  int32_t pad;
+};
+
+// An entry is one (sequence, KV head, stationary group) with a contiguous
+// range of streamed tiles ("steps").  Steps are split over CTAs by global
+// step index; the CTAs covering an entry are consecutive.
+struct Entry {
+  int32_t seq, g, grp, mode;
+  int32_t stat0;     // first stationary tile index (Q tile or K tile)
+  int32_t n_stat;    // stationary tiles in the group (1..4)
+  int32_t step0;     // first streamed tile index
+  int32_t n_steps;   // streamed tiles
+  int64_t sbase;     // global index of this entry's first step
+  int32_t unit_base; // partial-result slot of this entry's first unit
+  int32_t n_units;   // CTAs (units) covering the entry
+  int32_t first_cta;
+  int32_t pad[3];
+};
+
+struct PlanHeader {
+  uint32_t status;     // WAITS_DEV_* bits, cleared by the planner
+  int32_t n_e1, n_e2;  // entries per pass
+  int32_t n_u1, n_u2;  // units per pass
+  int32_t p1, p2;      // CTAs that own work per pass (<= grid)
+  int32_t pad0;
+  int64_t s1, s2;      // total steps per pass
+  int32_t pad[4];
+};
+
+// ------------------------------------------------------ workspace layout ---
+struct Layout {
+  size_t header, seqs, e1, e2, c1, c2, bias, part1, part2, total;
+  int64_t max_e1, max_e2, max_u1, max_u2;
+};
+
+__host__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Upper bounds that hold for every a, b (a = 0 activates every row).
+__host__ inline Layout make_layout(int64_t nseq, int64_t T, int64_t Hq, int64_t Hkv) {
+  Layout L{};
+  const int64_t G = Hq / Hkv;
+  const int64_t tokq = tokens_per_qtile((int)G);
+  L.max_e1 = Hkv * (T / (kMaxStat * tokq) + nseq);
+  L.max_e2 = Hkv * (T / (kMaxStat * kTile) + nseq);
+  L.max_u1 = L.max_e1 + kMaxGrid;
+  L.max_u2 = L.max_e2 + kMaxGrid;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  L.header = take(sizeof(PlanHeader));
+  L.seqs = take(sizeof(SeqInfo) * (size_t)nseq);
+  L.e1 = take(sizeof(Entry) * (size_t)L.max_e1);
+  L.e2 = take(sizeof(Entry) * (size_t)L.max_e2);
+  L.c1 = take(sizeof(uint32_t) * (size_t)L.max_e1);
+  L.c2 = take(sizeof(uint32_t) * (size_t)L.max_e2);
+  L.bias = take(sizeof(float) * (size_t)(Hq * T));
+  L.part1 = take(sizeof(float2) * (size_t)L.max_u1 * kMaxStat * kTile);
+  L.part2 = take(sizeof(float) * (size_t)L.max_u2 * kMaxStat * kTile);
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------ the curve ---
+// fp32 forgetting-curve weight (WAITS README, opening summary):
+// w = 1 / (1 + exp(-a (q - (N - b - 0.5)))), IEEE division, no flush to zero.
+__device__ inline float curve_weight(int q, int N, float a, int b) {
+  const float c = (float)N - (float)b - 0.5f;
+  const float t = -a * ((float)q - c);
+  return 1.0f / (1.0f + expf(t));
+}
+
+// First row whose fp32 weight is non-zero (N if none).  For a > 0 the weight
+// is non-decreasing in q, so a binary search finds it; a = 0 weights every
+// row by 1/2.
+__device__ inline int first_active_row(int N, float a, int b) {
+  if (N <= 0) return 0;
+  if (a == 0.0f) return 0;
+  if (!(curve_weight(N - 1, N, a, b) != 0.0f)) return N;
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {
+    const int mid = lo + (hi - lo) / 2;
+    if (curve_weight(mid, N, a, b) != 0.0f) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+// --------------------------------------------------------- block scans ---
+// Exclusive prefix sum over a block of kPlanThreads threads.
+__device__ inline int64_t block_exclusive_scan(int64_t v, int64_t* total, int64_t* sh /*[32]*/) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int64_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int64_t s = lane < nw ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int64_t y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    sh[lane] = s;  // inclusive warp totals
+  }
+  __syncthreads();
+  const int64_t before = (warp ? sh[warp - 1] : 0) + x - v;
+  *total = sh[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return before;
+}
+
+// -------------------------------------------------------- kernel params ---
+struct PlanArgs {
+  const int32_t* cu;
+  int nseq, T, max_seqlen, Hq, Hkv, G, tokq;
+  float a;
+  int b;
+  int grid;
+  PlanHeader* hdr;
+  SeqInfo* seqs;
+  Entry* e1;
+  Entry* e2;
+  uint32_t* c1;
+  uint32_t* c2;
+  int64_t max_e1, max_e2, max_u1, max_u2;
+  float* scores;  // zero-filled for sequences without active rows
+};
+
+struct PassArgs {
+  const uint16_t* Q;   // bf16 bits [T, Hq, d]
+  const uint16_t* K;   // bf16 bits [T, Hkv, d]
+  int T, Hq, Hkv, G, tokq, d;
+  float a;
+  int b;
+  float scale2;        // log2(e) / sqrt(d)
+  const PlanHeader* hdr;
+  const SeqInfo* seqs;
+  const Entry* e1;
+  const Entry* e2;
+  uint32_t* c1;
+  uint32_t* c2;
+  float* bias;         // [Hkv, T, G] log2 w - log2-sum-exp, active rows only
+  float2* part1;       // [units, 4, 128] (reference max, sum) in log2 units
+  float* part2;        // [units, 4, 128] partial column sums
+  float* scores;       // [Hkv, T]
+  uint32_t* status;
+};
+
+// Host-side launchers (one per translation unit).
+cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
+cudaError_t launch_score_passes(const PassArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int T,
+                          int Hkv, int R, int B, int32_t* idx, int32_t* kept_len,
+                          uint32_t* status, cudaStream_t s);
+cudaError_t launch_compact(const uint16_t* K, const uint16_t* V, const int32_t* cu,
+                           const int32_t* idx, const int32_t* kept_len, int nseq,
+                           int Hkv, int d, int B, uint16_t* Ko, uint16_t* Vo,
+                           uint32_t* status, cudaStream_t s);
+
+}  // namespace waits

@@ -1,0 +1,141 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+symbol its header declares, and rejects bad arguments on the host before any
+CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from prefill_eviction_scoring_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "waits.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(waits_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_bound_functions():
+    assert _declared() == sorted(_lib.SIGNATURES)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_strerror(lib):
+    assert lib.waits_abi_version() == 1
+    for st in range(8):
+        assert len(lib.waits_strerror(st)) >= 2
+    assert b"unknown" in lib.waits_strerror(99)
+
+
+FAKE = 0x100000   # never dereferenced: every call below fails validation
+
+
+def _shape(**kw):
+    d = dict(nseq=1, total_tokens=4096, max_seqlen=4096, num_q_heads=32,
+             num_kv_heads=8, head_dim=128, cu_seqlens=FAKE)
+    d.update(kw)
+    return _lib.Shape(**d)
+
+
+def _ws(lib, shape):
+    n = ctypes.c_size_t(0)
+    st = lib.waits_workspace_size(ctypes.byref(shape), ctypes.byref(n))
+    return st, n.value
+
+
+def test_workspace_size_host_only(lib):
+    st, n = _ws(lib, _shape())
+    assert st == 0 and n > 0
+    st2, n2 = _ws(lib, _shape(total_tokens=8192, max_seqlen=8192))
+    assert st2 == 0 and n2 > n
+    assert lib.waits_workspace_size(None, ctypes.byref(ctypes.c_size_t())) == 1
+    assert lib.waits_workspace_size(ctypes.byref(_shape()), None) == 1
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(nseq=0), 2), (dict(total_tokens=0), 2), (dict(num_q_heads=30), 2),
+    (dict(head_dim=96), 3), (dict(head_dim=256), 3),
+    (dict(num_q_heads=256, num_kv_heads=1), 3), (dict(max_seqlen=5000), 2),
+    (dict(cu_seqlens=0), 1), (dict(nseq=5000), 2)])
+def test_shape_errors(lib, kw, want):
+    assert _ws(lib, _shape(**kw))[0] == want
+
+
+def test_score_argument_errors(lib):
+    sh = _shape()
+    _, n = _ws(lib, sh)
+    W = 0x200000
+    call = lambda Q=FAKE, K=FAKE, a=1.0, b=16, s=FAKE, ws=W, nb=n: lib.waits_score(
+        ctypes.byref(sh), Q, K, a, b, s, ws, nb, None)
+    assert call(Q=None) == 1
+    assert call(K=None) == 1
+    assert call(s=None) == 1
+    assert call(Q=FAKE + 8) == 1                    # 16-byte alignment
+    assert call(a=-1.0) == 1
+    assert call(a=float("nan")) == 1
+    assert call(a=float("inf")) == 1
+    assert call(b=-1) == 1
+    assert call(ws=None) == 4
+    assert call(nb=n - 1) == 4
+    assert call(ws=W + 16) == 1                     # 256-byte alignment
+
+
+def test_select_compact_compress_errors(lib):
+    sh = _shape()
+    _, n = _ws(lib, sh)
+    assert lib.waits_select(ctypes.byref(sh), FAKE, 17, 16, FAKE, FAKE, None, 0, None) == 1
+    assert lib.waits_select(ctypes.byref(sh), FAKE, -1, 16, FAKE, FAKE, None, 0, None) == 1
+    assert lib.waits_select(ctypes.byref(sh), FAKE, 0, 0, FAKE, FAKE, None, 0, None) == 1
+    assert lib.waits_select(ctypes.byref(sh), None, 1, 16, FAKE, FAKE, None, 0, None) == 1
+    assert lib.waits_compact(ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE,
+                             None, 0, None) == 1
+    assert lib.waits_compact(ctypes.byref(sh), FAKE, FAKE + 4, FAKE, FAKE, 16, FAKE, FAKE,
+                             None, 0, None) == 1
+    assert lib.waits_compress(ctypes.byref(sh), FAKE, FAKE, FAKE, 1.0, 16, 32, 16, FAKE,
+                              FAKE, FAKE, FAKE, FAKE, 0x200000, n, None) == 1
+    assert lib.waits_compress(ctypes.byref(sh), FAKE, FAKE, FAKE, 1.0, 16, 16, 128, FAKE,
+                              FAKE, FAKE, FAKE, FAKE, 0x200000, 10, None) == 4
+
+
+def test_host_variant_validates_offsets(lib):
+    sh = _shape(nseq=2, total_tokens=100, max_seqlen=60)
+    _, n = _ws(lib, sh)
+    cu_bad = (ctypes.c_int32 * 3)(0, 70, 100)       # 70 > max_seqlen
+    cu_bad2 = (ctypes.c_int32 * 3)(0, 40, 90)       # does not end at T
+    bufs = _lib.DeviceBuffers(*([FAKE] * 9))
+    for cu in (cu_bad, cu_bad2):
+        st = lib.waits_compress_host(ctypes.byref(sh), cu, FAKE, FAKE, FAKE, 1.0, 16, 16,
+                                     128, FAKE, FAKE, FAKE, FAKE, ctypes.byref(bufs),
+                                     0x200000, n, None, None, None)
+        assert st == 2
+
+
+def test_status_read_needs_out_pointer(lib):
+    assert lib.waits_read_device_status(0x200000, 4096, None, None) == 1
+    assert lib.waits_read_device_status(None, 4096, None,
+                                        ctypes.byref(ctypes.c_uint32())) == 4
+
+
+def test_python_binding_fails_loudly_without_library(tmp_path):
+    saved = _lib._lib
+    _lib._lib = None
+    try:
+        with pytest.raises(_lib.WaitsLibraryError):
+            _lib.load(str(tmp_path / "missing.so"))
+    finally:
+        _lib._lib = saved

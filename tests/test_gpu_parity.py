@@ -1,0 +1,172 @@
+"""CUDA path vs the fp64 oracle, element by element, on seeded inputs that
+span several tiles and ragged tails (small enough for the oracle)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_parity import assert_scores_close, full_check, run_gpu
+from prefill_eviction_scoring_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("a,b", [(1.0, 16), (0.0, 16), (1e4, 1)])
+def test_tiny_config(a, b):
+    """N=512, 4 query heads on 1 KV head, d=64; a=1,b=16 plus the H2O and
+    TOVA limit actions."""
+    lay = wl.make_layer("tiny", device="cuda")
+    full_check(lay, a, b, 16, 128)
+
+
+@pytest.mark.parametrize("a,b", wl.WAITS_ACTIONS)
+def test_llama1b_shape_actions(a, b):
+    """1B-shaped heads (d=64, GQA 4, sink) at a length the oracle finishes
+    quickly, every README action."""
+    lay = wl.make_layer("llama1b", lens=(1100,), heads=(8, 2), device="cuda")
+    full_check(lay, a, b, 16, 128)
+
+
+@pytest.mark.parametrize("B", [128, 512])
+def test_llama8b_shape(B):
+    """8B-shaped heads (d=128, GQA 4) with sink and heavy hitters."""
+    lay = wl.make_layer("llama8b", lens=(2000,), heads=(8, 2), heavy_hitters=16,
+                        device="cuda")
+    full_check(lay, 1.0, 16, 16, B)
+
+
+def test_ragged_qwen_shape():
+    """Packed varlen batch with Qwen's G=7 grouping, lengths 1 and 129."""
+    lay = wl.make_layer("ragged", lens=(300, 129, 1, 700, 64), heads=(14, 2),
+                        device="cuda")
+    full_check(lay, 10.0, 16, 16, 128)
+
+
+def test_long_shape_dense_mode():
+    """a=0.01, b=128 activates ~9000 rows at full size; here about 1000 of
+    2500, enough for the stationary-K scheduling."""
+    lay = wl.make_layer("long", lens=(2500,), heads=(8, 2), heavy_hitters=32,
+                        device="cuda")
+    full_check(lay, 0.01, 128, 64, 256)
+
+
+@pytest.mark.parametrize("case", [
+    dict(lens=(50,), a=1.0, b=16, R=16, B=128),         # N < tile, N <= B
+    dict(lens=(129,), a=1.0, b=16, R=16, B=128),        # one past B
+    dict(lens=(700,), a=1.0, b=16, R=0, B=64),          # R = 0
+    dict(lens=(700,), a=1.0, b=16, R=64, B=64),         # R = B
+    dict(lens=(512,), a=1.0, b=600, R=16, B=128),       # b >= N
+    dict(lens=(400,), a=1e4, b=0, R=16, B=128),         # no active row at all
+    dict(lens=(1, 1, 300), a=0.0, b=1, R=2, B=4),       # one-token sequences
+    dict(lens=(1000,), a=0.3, b=40, R=8, B=300),
+])
+@pytest.mark.parametrize("d", [64, 128])
+def test_edge_cases(case, d):
+    lay = wl.random_layer(case["lens"], 8, 2, d, seed=77 + d, device="cuda")
+    full_check(lay, case["a"], case["b"], case["R"], case["B"])
+
+
+def test_exact_ties_bit_exact():
+    """a=1e4, b=1 and a zero last query: every score is exactly G/N and the
+    kept pool is the lowest indices."""
+    N, G = 256, 4
+    lay = wl.random_layer((N,), 8, 2, 128, seed=5, device="cuda")
+    lay.Q[N - 1] = 0
+    gpu = run_gpu(lay, 1e4, 1, 16, 64)
+    assert np.all(gpu["scores"] == G / N)
+    want = list(range(48)) + list(range(N - 16, N))
+    for g in range(2):
+        assert gpu["idx"][0, g].tolist() == want
+
+
+def test_zero_keys_closed_form():
+    """K = 0: P[q,k] = 1/(q+1), so at a=0 the scores are (G/2)(H_N - H_k)."""
+    N, G = 600, 4
+    lay = wl.random_layer((N,), 8, 2, 128, seed=6, device="cuda")
+    lay.K.zero_()
+    gpu = run_gpu(lay, 0.0, 1, 16, 128)
+    H = np.concatenate([[0.0], np.cumsum(1.0 / np.arange(1, N + 1))])
+    want = 0.5 * G * (H[N] - H[:N])
+    for g in range(2):
+        assert_scores_close(gpu["scores"][g:g + 1], want[None, :])
+
+
+def test_sum_identity():
+    """Each query row's P sums to 1: sum_k s[g,k] = G * sum_q w[q]."""
+    lay = wl.make_layer("llama8b", lens=(3000, 1000), heads=(8, 2), device="cuda")
+    gpu = run_gpu(lay, 0.05, 30, 16, 128)
+    cu = lay.cu_seqlens.cpu().numpy()
+    for i in range(2):
+        N = cu[i + 1] - cu[i]
+        w = oracle.forgetting_curve(np.arange(N), N, 0.05, 30)
+        for g in range(2):
+            tot = gpu["scores"][g, cu[i]:cu[i + 1]].sum()
+            assert abs(tot - 4 * w.sum()) <= 1e-5 * 4 * w.sum()
+
+
+def test_deterministic_bits():
+    lay = wl.make_layer("llama8b", lens=(1500, 900), heads=(8, 2), device="cuda")
+    a = run_gpu(lay, 0.02, 64, 16, 128)
+    b = run_gpu(lay, 0.02, 64, 16, 128)
+    assert torch.equal(a["raw_scores"].view(torch.int32), b["raw_scores"].view(torch.int32))
+    assert np.array_equal(a["idx"], b["idx"])
+
+
+def test_separate_calls_equal_fused():
+    """waits_score, waits_select and waits_compact called one by one give
+    the same bits as waits_compress."""
+    from prefill_eviction_scoring_b200 import api
+    lay = wl.make_layer("ragged", lens=(400, 250), heads=(7, 1), device="cuda")
+    s = api.score(lay.Q, lay.K, lay.cu_seqlens, sigmoid_a=1.0, window=16)
+    idx, kept = api.select(s, lay.cu_seqlens, recent_budget=16, budget=128)
+    Ko, Vo = api.compact(lay.K, lay.V, lay.cu_seqlens, idx, kept)
+    Ko2, Vo2, idx2, kept2, s2 = api.compress(lay.Q, lay.K, lay.V, lay.cu_seqlens, sigmoid_a=1.0,
+                                             window=16, recent_budget=16, budget=128)
+    torch.cuda.synchronize()
+    assert torch.equal(s.view(torch.int32), s2.view(torch.int32))
+    assert torch.equal(idx, idx2) and torch.equal(kept, kept2)
+    assert torch.equal(Ko.view(torch.int16), Ko2.view(torch.int16))
+    assert torch.equal(Vo.view(torch.int16), Vo2.view(torch.int16))
+
+
+def test_bad_seqlens_flagged_not_faulting():
+    """Malformed cu_seqlens are caught on the device: status bit set, no work."""
+    from prefill_eviction_scoring_b200 import Compressor, _lib
+    lay = wl.random_layer((300, 200), 8, 2, 64, seed=9, device="cuda")
+    bad = torch.tensor([0, 350, 500], dtype=torch.int32, device="cuda")   # 350 > max 300
+    c = Compressor(bad, 500, 300, 8, 2, 64, 128)
+    c(lay.Q, lay.K, lay.V, 1.0, 16, 16)
+    torch.cuda.synchronize()
+    assert c.device_status() & _lib.DEV_BAD_SEQLENS
+
+
+def test_compact_bad_index_flagged():
+    from prefill_eviction_scoring_b200 import api, _lib
+    lay = wl.random_layer((100,), 8, 2, 128, seed=10, device="cuda")
+    idx = torch.arange(16, dtype=torch.int32, device="cuda").view(1, 1, 16).repeat(1, 2, 1)
+    idx[0, 1, 3] = 100        # == N: out of range
+    kept = torch.tensor([16], dtype=torch.int32, device="cuda")
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    Ko, Vo = api.compact(lay.K, lay.V, lay.cu_seqlens, idx, kept, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) & _lib.DEV_BAD_INDEX
+    assert torch.all(Ko[0, 1, 3] == 0)
+    assert torch.equal(Ko[0, 0], lay.K[:16, 0])
+
+
+def test_host_buffer_entry_point():
+    """waits_compress_host gives the same result as the device entry point."""
+    from prefill_eviction_scoring_b200 import HostCompressor
+    lay = wl.make_layer("ragged", lens=(900, 333), heads=(14, 2), device="cuda")
+    gpu = run_gpu(lay, 1.0, 16, 16, 128, canary=False)
+    hc = HostCompressor(lay.cu_seqlens.cpu(), 14, 2, 128, 128)
+    Qh, Kh, Vh = (t.cpu().pin_memory() for t in (lay.Q, lay.K, lay.V))
+    Ko, Vo, idx, kept = hc(Qh, Kh, Vh, 1.0, 16, 16)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.numpy(), gpu["idx"])
+    assert np.array_equal(Ko.view(torch.int16).numpy(), gpu["Ko"])
+    assert np.array_equal(Vo.view(torch.int16).numpy(), gpu["Vo"])
+    kv = 1233 * 2 * 128 * 2 * 2
+    q_active = 2 * 120 * 14 * 128 * 2          # ~b + 90/a rows per sequence
+    assert kv < hc.h2d_bytes < kv + q_active + 4096   # only the active Q rows
