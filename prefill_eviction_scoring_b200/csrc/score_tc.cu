@@ -27,15 +27,17 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kEpiWarps = 4;
-constexpr int kThreads = (kEpiWarps + 2) * 32;
-constexpr int kProducerWarp = kEpiWarps;
-constexpr int kMmaWarp = kEpiWarps + 1;
-constexpr int kTmemBufs = 4;
+constexpr int kWGs = 2;                              // epilogue warpgroups
+constexpr int kEpiThreads = kWGs * 128;
+constexpr int kThreads = kEpiThreads + 64;           // + producer warp + MMA warp
+constexpr int kProducerWarp = kWGs * 4;
+constexpr int kMmaWarp = kProducerWarp + 1;
+constexpr int kTmemBufs = 2 * kWGs;                  // two 128-column buffers per WG
 constexpr int kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s after an abort
-constexpr int kEpiBar = 1;                          // named barrier of warps 0-3
+constexpr int kBarWG0 = 1;                           // named barriers: 1, 2 per WG,
+constexpr int kBarAll = 3;                           // 3 for both WGs
 
 template <int D>
 struct Cfg {
@@ -44,15 +46,20 @@ struct Cfg {
   static constexpr int kTileBytes = kSub * kSubBytes;
   static constexpr int kStages = D == 128 ? 2 : 4;
   static constexpr int kKSteps = D / 16;
+  static constexpr size_t kFloats = kMaxStat * kTile            // stationary Q biases
+                                    + kWGs * 2 * kTile           // streamed Q biases
+                                    + 2 * kWGs * kMaxStat * kTile;  // per-WG state
   static constexpr size_t kSmem = 1024 + (size_t)(kMaxStat + kStages) * kTileBytes +
-                                  (kMaxStat + 2) * kTile * sizeof(float) + 256;
+                                  kFloats * sizeof(float) + 256;
 };
 
 struct Smem {
   uint8_t* stat;
   uint8_t* strm;
   float* bias_stat;  // [4][128]
-  float* bias_strm;  // [2][128]
+  float* bias_strm;  // [WG][2][128]
+  float* st_m;       // [WG][4][128] reference max (pass 1)
+  float* st_l;       // [WG][4][128] running sum (pass 1) / column sum (pass 2)
   uint64_t* full;
   uint64_t* empty;
   uint64_t* stat_full;
@@ -75,7 +82,9 @@ __device__ Smem carve(uint8_t* raw) {
   s.strm = s.stat + kMaxStat * C::kTileBytes;
   s.bias_stat = reinterpret_cast<float*>(s.strm + C::kStages * C::kTileBytes);
   s.bias_strm = s.bias_stat + kMaxStat * kTile;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.bias_strm + 2 * kTile);
+  s.st_m = s.bias_strm + kWGs * 2 * kTile;
+  s.st_l = s.st_m + kWGs * kMaxStat * kTile;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.st_l + kWGs * kMaxStat * kTile);
   s.full = bars;
   s.empty = s.full + C::kStages;
   s.stat_full = s.empty + C::kStages;
@@ -93,6 +102,12 @@ __device__ inline float u2f(uint32_t v) { return __uint_as_float(v); }
 
 // Streamed / stationary operand kinds per mode.
 __device__ inline bool stat_is_q(int mode) { return mode != kModeP2K; }
+
+// (Q tile, K tile) of the pair (streamed tile o, stationary slot i).
+__device__ inline void pair_tiles(const Entry& e, int o, int i, int& j, int& kt) {
+  j = e.mode == kModeP2K ? o : e.stat0 + i;
+  kt = e.mode == kModeP2K ? e.stat0 + i : o;
+}
 
 // ------------------------------------------------------------ producer ---
 template <int D>
@@ -157,13 +172,17 @@ out:
 }
 
 // ---------------------------------------------------------- MMA issuer ---
+// Streamed tiles are taken two at a time; the pairs of the first go to
+// epilogue warpgroup 0, those of the second to warpgroup 1, interleaved so
+// both groups always have work.  Each group owns two TMEM buffers.
 template <int D>
 __device__ void mma_issuer(const PassArgs& p, const Smem& s, const Entry* E, UnitIter it,
                            uint32_t tmem) {
   using C = Cfg<D>;
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
-  int stage = 0, buf = 0;
-  uint32_t sph = 0, uph = 0, bph = 0;
+  int stage = 0;
+  uint32_t sph = 0, uph = 0;
+  uint32_t kpair[kWGs] = {0, 0};
   const uint32_t stat0 = smem_addr(s.stat), strm0 = smem_addr(s.strm);
   int ei, st0, st1, unit;
   while (it.next(ei, st0, st1, unit)) {
@@ -172,34 +191,44 @@ __device__ void mma_issuer(const PassArgs& p, const Smem& s, const Entry* E, Uni
     if (!mbar_wait(s.stat_full, uph, s.abort, p.status, kWaitLimitNs)) goto out;
     uph ^= 1u;
     tc_fence_after();
-    for (int st = st0; st < st1; ++st) {
-      const int o = e.step0 + st;
-      if (!mbar_wait(&s.full[stage], sph, s.abort, p.status, kWaitLimitNs)) goto out;
-      tc_fence_after();
-      const uint32_t sa = strm0 + stage * C::kTileBytes;
-      for (int i = 0; i < e.n_stat; ++i) {
-        const int j = e.mode == kModeP2K ? o : e.stat0 + i;
-        const int kt = e.mode == kModeP2K ? e.stat0 + i : o;
-        if (!pair_live(si, j, kt, p.tokq)) continue;
-        if (!mbar_wait(&s.tempty[buf], bph ^ 1u, s.abort, p.status, kWaitLimitNs)) goto out;
-        tc_fence_after();
-        const uint32_t ta = stat0 + i * C::kTileBytes;
-        // P1: A = Q (stationary), B = K (streamed); P2Q: A = K (streamed),
-        // B = Q (stationary); P2K: A = K (stationary), B = Q (streamed).
-        const uint32_t a_base = e.mode == kModeP2Q ? sa : ta;
-        const uint32_t b_base = e.mode == kModeP2Q ? ta : sa;
-        const uint32_t d_tmem = tmem + (uint32_t)(buf * kTile);
-#pragma unroll
-        for (int k = 0; k < C::kKSteps; ++k) {
-          const uint32_t off = (uint32_t)((k >> 2) * C::kSubBytes + (k & 3) * 32);
-          mma_bf16(d_tmem, sdesc_kmajor_sw128(a_base + off), sdesc_kmajor_sw128(b_base + off),
-                   idesc, k > 0 ? 1u : 0u);
-        }
-        mma_commit(&s.tfull[buf]);
-        if (++buf == kTmemBufs) { buf = 0; bph ^= 1u; }
+    const int n = st1 - st0;
+    for (int ls = 0; ls < n; ls += kWGs) {
+      const int nw = n - ls < kWGs ? n - ls : kWGs;     // streamed tiles this round
+      int stg[kWGs];
+      for (int w = 0; w < nw; ++w) {
+        stg[w] = stage;
+        if (!mbar_wait(&s.full[stage], sph, s.abort, p.status, kWaitLimitNs)) goto out;
+        if (++stage == C::kStages) { stage = 0; sph ^= 1u; }
       }
-      mma_commit(&s.empty[stage]);
-      if (++stage == C::kStages) { stage = 0; sph ^= 1u; }
+      tc_fence_after();
+      for (int i = 0; i < e.n_stat; ++i) {
+        for (int w = 0; w < nw; ++w) {
+          const int o = e.step0 + st0 + ls + w;
+          int j, kt;
+          pair_tiles(e, o, i, j, kt);
+          if (!pair_live(si, j, kt, p.tokq)) continue;
+          const int buf = 2 * w + (int)(kpair[w] & 1u);
+          const uint32_t ph = (kpair[w] >> 1) & 1u;
+          if (!mbar_wait(&s.tempty[buf], ph ^ 1u, s.abort, p.status, kWaitLimitNs)) goto out;
+          tc_fence_after();
+          const uint32_t sa = strm0 + stg[w] * C::kTileBytes;
+          const uint32_t ta = stat0 + i * C::kTileBytes;
+          // P1: A = Q (stationary), B = K (streamed); P2Q: A = K (streamed),
+          // B = Q (stationary); P2K: A = K (stationary), B = Q (streamed).
+          const uint32_t a_base = e.mode == kModeP2Q ? sa : ta;
+          const uint32_t b_base = e.mode == kModeP2Q ? ta : sa;
+          const uint32_t d_tmem = tmem + (uint32_t)(buf * kTile);
+#pragma unroll
+          for (int k = 0; k < C::kKSteps; ++k) {
+            const uint32_t off = (uint32_t)((k >> 2) * C::kSubBytes + (k & 3) * 32);
+            mma_bf16(d_tmem, sdesc_kmajor_sw128(a_base + off),
+                     sdesc_kmajor_sw128(b_base + off), idesc, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&s.tfull[buf]);
+          ++kpair[w];
+        }
+      }
+      for (int w = 0; w < nw; ++w) mma_commit(&s.empty[stg[w]]);
     }
     mma_commit(s.stat_empty);
   }
@@ -211,111 +240,104 @@ out:
 }
 
 // ------------------------------------------------------------ epilogue ---
-// Load 32 TMEM columns of this warp's lanes; the wait names the registers so
-// no use of them can be scheduled before the data has arrived.
-struct Chunk {
-  uint32_t r[32];
-  __device__ void load(uint32_t taddr) { tmem_ld32(taddr, r); }
+// 128 accumulator columns of this thread's TMEM lane.  The wait names every
+// register so no use of them can be scheduled before the data has arrived.
+struct Cols {
+  uint32_t r[128];
+  __device__ void load(uint32_t taddr) {
+    uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+    uint32_t(&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+    uint32_t(&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
+    uint32_t(&d)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
+    tmem_ld32(taddr, a);
+    tmem_ld32(taddr + 32, b);
+    tmem_ld32(taddr + 64, c);
+    tmem_ld32(taddr + 96, d);
+  }
   __device__ void wait() {
+#define W8(b) "+r"(r[b]), "+r"(r[b + 1]), "+r"(r[b + 2]), "+r"(r[b + 3]), "+r"(r[b + 4]), \
+              "+r"(r[b + 5]), "+r"(r[b + 6]), "+r"(r[b + 7])
     asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]),
-                   "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
-                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]),
-                   "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 : W8(0), W8(8), W8(16), W8(24), W8(32), W8(40), W8(48), W8(56), W8(64), W8(72),
+                   W8(80), W8(88), W8(96), W8(104), W8(112), W8(120)
                  :
                  : "memory");
+#undef W8
   }
 };
 
-// Pass 1, one chunk of 32 keys for this thread's row: adds
-// sum 2^(v*scale2 - mref) over the valid keys (c < nv) to *acc (relative to
-// mref), moving mref up when the running sum would leave the safe range.
-__device__ inline void p1_chunk(const Chunk& ch, int cbase, int nv, float scale2, float& mref,
-                                float& lsum, float& acc) {
-  if (cbase >= nv) return;
-  const bool masked = cbase + 32 > nv;
-  if (mref == -INFINITY) {
+// Pass 1, one 128-key tile of this thread's row (keys c < nv are causal):
+// l += sum_c 2^(v_c*scale2 - m), m = first maximum seen, moved up only when
+// the running sum would leave the safe fp32 range.
+__device__ inline void p1_pair(const Cols& v, int nv, float sc, float& m, float& l) {
+  if (nv <= 0) return;
+  if (m == -INFINITY) {
     float mx = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (!masked || cbase + j < nv) mx = fmaxf(mx, u2f(ch.r[j]) * scale2);
-    mref = mx;
+    for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, c < nv ? u2f(v.r[c]) * sc : -INFINITY);
+    m = mx;
   }
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-  if (!masked) {
+  const float nm = -m;
+  float a[8];
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      s0 += ex2_approx(fmaf(u2f(ch.r[j + 0]), scale2, -mref));
-      s1 += ex2_approx(fmaf(u2f(ch.r[j + 1]), scale2, -mref));
-      s2 += ex2_approx(fmaf(u2f(ch.r[j + 2]), scale2, -mref));
-      s3 += ex2_approx(fmaf(u2f(ch.r[j + 3]), scale2, -mref));
-    }
-  } else {
+  for (int k = 0; k < 8; ++k) a[k] = 0.f;
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      s0 += cbase + j + 0 < nv ? ex2_approx(fmaf(u2f(ch.r[j + 0]), scale2, -mref)) : 0.f;
-      s1 += cbase + j + 1 < nv ? ex2_approx(fmaf(u2f(ch.r[j + 1]), scale2, -mref)) : 0.f;
-      s2 += cbase + j + 2 < nv ? ex2_approx(fmaf(u2f(ch.r[j + 2]), scale2, -mref)) : 0.f;
-      s3 += cbase + j + 3 < nv ? ex2_approx(fmaf(u2f(ch.r[j + 3]), scale2, -mref)) : 0.f;
-    }
+  for (int c = 0; c < kTile; ++c) {
+    const float x = fmaf(u2f(v.r[c]), sc, nm);
+    a[c & 7] += ex2_approx(c < nv ? x : -INFINITY);
   }
-  const float cs = (s0 + s1) + (s2 + s3);
-  if (lsum + acc + cs <= kRebaseLimit) {
-    acc += cs;
+  const float t = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+  if (l + t <= kRebaseLimit) {
+    l += t;
     return;
   }
-  // a value far above the reference: rebase on this chunk's maximum
-  float mx = mref;
+  // a value far above the reference: rebase on this tile's maximum
+  float mx = m;
 #pragma unroll
-  for (int j = 0; j < 32; ++j)
-    if (!masked || cbase + j < nv) mx = fmaxf(mx, u2f(ch.r[j]) * scale2);
-  const float f = ex2_approx(mref - mx);
-  lsum *= f;
-  acc *= f;
-  float t = 0.f;
+  for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, c < nv ? u2f(v.r[c]) * sc : -INFINITY);
+  float t2 = 0.f;
 #pragma unroll
-  for (int j = 0; j < 32; ++j)
-    if (!masked || cbase + j < nv) t += ex2_approx(fmaf(u2f(ch.r[j]), scale2, -mx));
-  acc += t;
-  mref = mx;
+  for (int c = 0; c < kTile; ++c) {
+    const float x = fmaf(u2f(v.r[c]), sc, -mx);
+    t2 += ex2_approx(c < nv ? x : -INFINITY);
+  }
+  l = l * ex2_approx(m - mx) + t2;
+  m = mx;
 }
 
-// Pass 2, one chunk of 32 query columns for this thread's key: adds
-// sum 2^(v*scale2 + bias[c]) over columns c in [c0, 128).
-__device__ inline float p2_chunk(const Chunk& ch, int cbase, int c0, float scale2,
-                                 const float* bias) {
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-  const float4* b4 = reinterpret_cast<const float4*>(bias + cbase);
-  if (c0 <= cbase) {
+// Pass 2, one 128-row Q tile for this thread's key: sum over columns
+// c in [c_lo, ncols) of 2^(v_c*scale2 + bias_c).
+__device__ inline float p2_pair(const Cols& v, int c_lo, int ncols, float sc, const float* bias) {
+  float a[8];
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      const float4 b = b4[j / 4];
-      s0 += ex2_approx(fmaf(u2f(ch.r[j + 0]), scale2, b.x));
-      s1 += ex2_approx(fmaf(u2f(ch.r[j + 1]), scale2, b.y));
-      s2 += ex2_approx(fmaf(u2f(ch.r[j + 2]), scale2, b.z));
-      s3 += ex2_approx(fmaf(u2f(ch.r[j + 3]), scale2, b.w));
-    }
-  } else {
+  for (int k = 0; k < 8; ++k) a[k] = 0.f;
+  const float4* b4 = reinterpret_cast<const float4*>(bias);
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      const float4 b = b4[j / 4];
-      s0 += cbase + j + 0 >= c0 ? ex2_approx(fmaf(u2f(ch.r[j + 0]), scale2, b.x)) : 0.f;
-      s1 += cbase + j + 1 >= c0 ? ex2_approx(fmaf(u2f(ch.r[j + 1]), scale2, b.y)) : 0.f;
-      s2 += cbase + j + 2 >= c0 ? ex2_approx(fmaf(u2f(ch.r[j + 2]), scale2, b.z)) : 0.f;
-      s3 += cbase + j + 3 >= c0 ? ex2_approx(fmaf(u2f(ch.r[j + 3]), scale2, b.w)) : 0.f;
+  for (int cb = 0; cb < kTile; cb += 32) {
+    if (cb < ncols) {
+#pragma unroll
+      for (int c = cb; c < cb + 32; c += 4) {
+        const float4 b = b4[c / 4];
+        const float x0 = fmaf(u2f(v.r[c + 0]), sc, b.x);
+        const float x1 = fmaf(u2f(v.r[c + 1]), sc, b.y);
+        const float x2 = fmaf(u2f(v.r[c + 2]), sc, b.z);
+        const float x3 = fmaf(u2f(v.r[c + 3]), sc, b.w);
+        a[(c + 0) & 7] += ex2_approx(c + 0 >= c_lo ? x0 : -INFINITY);
+        a[(c + 1) & 7] += ex2_approx(c + 1 >= c_lo ? x1 : -INFINITY);
+        a[(c + 2) & 7] += ex2_approx(c + 2 >= c_lo ? x2 : -INFINITY);
+        a[(c + 3) & 7] += ex2_approx(c + 3 >= c_lo ? x3 : -INFINITY);
+      }
     }
   }
-  return (s0 + s1) + (s2 + s3);
+  return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
-__device__ inline void epi_sync() {
+__device__ inline void bar_sync(int id, int n) {
   __syncwarp();
-  named_bar_sync(kEpiBar, kEpiWarps * 32);
+  named_bar_sync(id, n);
 }
-// Barrier of warps 0-3 that also ORs `v` over them (a uniform answer).
-__device__ inline bool epi_vote_or(bool v) {
+// Named barrier that also ORs `v` over its threads (a uniform answer).
+__device__ inline bool bar_vote_or(int id, int n, bool v) {
   __syncwarp();
   uint32_t r;
   asm volatile(
@@ -324,7 +346,7 @@ __device__ inline bool epi_vote_or(bool v) {
       "bar.red.or.pred q, %2, %3, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)v), "r"(kEpiBar), "r"(kEpiWarps * 32)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
       : "memory");
   return r != 0;
 }
@@ -343,94 +365,84 @@ __device__ void write_row_bias(const PassArgs& p, const SeqInfo& si, int g, int 
   p.bias[((size_t)g * p.T + si.start + tok) * p.G + hg] = w > 0.f ? log2f(w) - lse2 : -INFINITY;
 }
 
+// Merge two (reference max, sum) pairs of the same row.
+__device__ inline float2 lse_merge(float2 x, float2 y) {
+  if (!(y.y > 0.f)) return x;
+  if (!(x.y > 0.f)) return y;
+  const float M = fmaxf(x.x, y.x);
+  return make_float2(M, x.y * ex2_approx(x.x - M) + y.y * ex2_approx(y.x - M));
+}
+
 template <int D>
 __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitIter it,
-                         uint32_t tmem, bool pass1) {
-  const int t = threadIdx.x;                 // TMEM lane == row (pass 1) / key (pass 2)
-  const int warp = t >> 5, lane = t & 31;
-  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-  int buf = 0, sstep = 0;
-  uint32_t bph = 0;
-  bool ok = true;   // false after a timeout: keep every barrier, skip the work
+                         uint32_t tmem) {
+  const int tid = threadIdx.x;               // 0..255
+  const int wg = tid >> 7;                    // warpgroup
+  const int t = tid & 127;                    // TMEM lane == row (pass 1) / key (pass 2)
+  const int lane = tid & 31;
+  const uint32_t lane_addr = tmem + ((uint32_t)((t >> 5) * 32) << 16);
+  const int bar_wg = kBarWG0 + wg;
+  float* my_m = s.st_m + wg * kMaxStat * kTile + t;
+  float* my_l = s.st_l + wg * kMaxStat * kTile + t;
+  uint32_t kp = 0;          // pairs consumed by this warpgroup
+  int sstep = 0;            // streamed steps consumed by this warpgroup
+  bool ok = true;           // false after a timeout: keep every barrier, skip the work
   int ei, st0, st1, unit;
   while (it.next(ei, st0, st1, unit)) {
     const Entry e = E[ei];
     const SeqInfo si = p.seqs[e.seq];
     const int g = e.g;
-    float mref[kMaxStat], lsum[kMaxStat], acc[kMaxStat];
-#pragma unroll
-    for (int i = 0; i < kMaxStat; ++i) { mref[i] = -INFINITY; lsum[i] = 0.f; acc[i] = 0.f; }
+    for (int i = 0; i < kMaxStat; ++i) { my_m[i * kTile] = -INFINITY; my_l[i * kTile] = 0.f; }
+    bar_sync(kBarAll, kEpiThreads);   // previous unit fully merged
     if (e.mode == kModeP2Q) {
-      epi_sync();
-      for (int i = 0; i < e.n_stat; ++i) s.bias_stat[i * kTile + t] = qrow_bias(p, si, g, e.stat0 + i, t);
-      epi_sync();
+      for (int i = wg; i < e.n_stat; i += kWGs)
+        s.bias_stat[i * kTile + t] = qrow_bias(p, si, g, e.stat0 + i, t);
+      bar_sync(kBarAll, kEpiThreads);
     }
-    for (int st = st0; st < st1; ++st) {
-      const int o = e.step0 + st;
-      float* bias_o = s.bias_strm + (sstep & 1) * kTile;
+    const int n = st1 - st0;
+    for (int ls = wg; ls < n; ls += kWGs) {
+      const int o = e.step0 + st0 + ls;
+      float* bias_o = s.bias_strm + (wg * 2 + (sstep & 1)) * kTile;
+      ++sstep;
       if (e.mode == kModeP2K) {
         bias_o[t] = qrow_bias(p, si, g, o, t);
-        epi_sync();
+        bar_sync(bar_wg, 128);
       }
-      ++sstep;
       float col = 0.f;
-#pragma unroll
-      for (int i = 0; i < kMaxStat; ++i) {
-        if (i >= e.n_stat) break;
-        const int j = e.mode == kModeP2K ? o : e.stat0 + i;
-        const int kt = e.mode == kModeP2K ? e.stat0 + i : o;
+      for (int i = 0; i < e.n_stat; ++i) {
+        int j, kt;
+        pair_tiles(e, o, i, j, kt);
         if (!pair_live(si, j, kt, p.tokq)) continue;
-        if (ok && !mbar_wait(&s.tfull[buf], bph, s.abort, p.status, kWaitLimitNs)) ok = false;
-        if (!ok) { if (++buf == kTmemBufs) { buf = 0; bph ^= 1u; } continue; }
+        const int buf = 2 * wg + (int)(kp & 1u);
+        const uint32_t ph = (kp >> 1) & 1u;
+        ++kp;
+        if (ok && !mbar_wait(&s.tfull[buf], ph, s.abort, p.status, kWaitLimitNs)) ok = false;
+        if (!ok) continue;
         tc_fence_after();
-        const uint32_t ta = lane_addr + (uint32_t)(buf * kTile);
-        Chunk c0, c1;
+        Cols v;
+        v.load(lane_addr + (uint32_t)(buf * kTile));
+        v.wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.tempty[buf]);
         if (e.mode == kModeP1) {
           const int tok = si.q0 + j * p.tokq + t / p.G;
           const bool row_ok = t < p.tokq * p.G && tok < si.len;
           int nv = row_ok ? tok - kt * kTile + 1 : 0;
-          nv = nv > kTile ? kTile : (nv < 0 ? 0 : nv);
-          float a2 = 0.f;
-          c0.load(ta); c0.wait();
-          c1.load(ta + 32);
-          p1_chunk(c0, 0, nv, p.scale2, mref[i], lsum[i], a2);
-          __syncwarp(); c1.wait();
-          c0.load(ta + 64);
-          p1_chunk(c1, 32, nv, p.scale2, mref[i], lsum[i], a2);
-          __syncwarp(); c0.wait();
-          c1.load(ta + 96);
-          p1_chunk(c0, 64, nv, p.scale2, mref[i], lsum[i], a2);
-          __syncwarp(); c1.wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s.tempty[buf]);
-          p1_chunk(c1, 96, nv, p.scale2, mref[i], lsum[i], a2);
-          lsum[i] += a2;
+          nv = nv > kTile ? kTile : nv;
+          float m = my_m[i * kTile], l = my_l[i * kTile];
+          p1_pair(v, nv, p.scale2, m, l);
+          my_m[i * kTile] = m;
+          my_l[i * kTile] = l;
         } else {
           const int key = kt * kTile + t;
           const int f = si.q0 + j * p.tokq;
-          const int cmin = key > f ? (key - f) * p.G : 0;
-          const int c_lo = cmin > kTile ? kTile : cmin;
+          const int c_lo = key > f ? min((key - f) * p.G, kTile) : 0;
           const int ncols = min(p.tokq, si.len - f) * p.G;   // valid columns (uniform)
           const float* bias = e.mode == kModeP2K ? bias_o : s.bias_stat + i * kTile;
-          float a2 = 0.f;
-          c0.load(ta); c0.wait();
-          c1.load(ta + 32);
-          if (0 < ncols) a2 += p2_chunk(c0, 0, c_lo, p.scale2, bias);
-          __syncwarp(); c1.wait();
-          c0.load(ta + 64);
-          if (32 < ncols) a2 += p2_chunk(c1, 32, c_lo, p.scale2, bias);
-          __syncwarp(); c0.wait();
-          c1.load(ta + 96);
-          if (64 < ncols) a2 += p2_chunk(c0, 64, c_lo, p.scale2, bias);
-          __syncwarp(); c1.wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s.tempty[buf]);
-          if (96 < ncols) a2 += p2_chunk(c1, 96, c_lo, p.scale2, bias);
-          if (e.mode == kModeP2K) acc[i] += a2; else col += a2;
+          const float a2 = p2_pair(v, c_lo, ncols, p.scale2, bias);
+          if (e.mode == kModeP2K) my_l[i * kTile] += a2; else col += a2;
         }
-        if (++buf == kTmemBufs) { buf = 0; bph ^= 1u; }
       }
       if (e.mode == kModeP2Q && ok) {
         const int key = o * kTile + t;
@@ -438,61 +450,64 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
       }
     }
 
-    // ---- unit results (skipped by all epilogue threads together after a timeout)
-    if (epi_vote_or(!ok || *s.abort)) { ok = false; continue; }
+    // ---- unit results: both warpgroups' partial states are merged by WG 0
+    const bool fail = bar_vote_or(kBarAll, kEpiThreads, !ok || *s.abort);
+    float2 st[kMaxStat];
+    if (!fail && wg == 0 && e.mode != kModeP2Q) {
+#pragma unroll
+      for (int i = 0; i < kMaxStat; ++i) {
+        const float2 a = make_float2(my_m[i * kTile], my_l[i * kTile]);
+        const float2 b = make_float2(my_m[kMaxStat * kTile + i * kTile],
+                                     my_l[kMaxStat * kTile + i * kTile]);
+        st[i] = e.mode == kModeP1 ? lse_merge(a, b) : make_float2(0.f, a.y + b.y);
+      }
+    }
+    if (fail) { ok = false; continue; }
+    if (wg != 0 || e.mode == kModeP2Q) continue;
     if (e.mode == kModeP1) {
       if (e.n_units == 1) {
 #pragma unroll
         for (int i = 0; i < kMaxStat; ++i) {
-          if (i >= e.n_stat) break;
           const int tok = si.q0 + (e.stat0 + i) * p.tokq + t / p.G;
-          if (t < p.tokq * p.G && tok < si.len)
-            write_row_bias(p, si, g, tok, t % p.G, mref[i] + log2f(lsum[i]));
+          if (i < e.n_stat && t < p.tokq * p.G && tok < si.len)
+            write_row_bias(p, si, g, tok, t % p.G, st[i].x + log2f(st[i].y));
         }
       } else {
 #pragma unroll
         for (int i = 0; i < kMaxStat; ++i)
-          if (i < e.n_stat)
-            p.part1[((size_t)unit * kMaxStat + i) * kTile + t] = make_float2(mref[i], lsum[i]);
+          if (i < e.n_stat) p.part1[((size_t)unit * kMaxStat + i) * kTile + t] = st[i];
         __threadfence();
-        epi_sync();
+        bar_sync(kBarWG0, 128);
         if (t == 0) *s.last = atomicAdd(&p.c1[ei], 1u) == (uint32_t)(e.n_units - 1);
-        epi_sync();
+        bar_sync(kBarWG0, 128);
         if (*s.last) {
           __threadfence();
           for (int i = 0; i < e.n_stat; ++i) {
             const int tok = si.q0 + (e.stat0 + i) * p.tokq + t / p.G;
             if (t >= p.tokq * p.G || tok >= si.len) continue;
             const float2* parts = p.part1 + ((size_t)e.unit_base * kMaxStat + i) * kTile + t;
-            float M = -INFINITY;
-            for (int u = 0; u < e.n_units; ++u) {
-              const float2 v = __ldcg(parts + (size_t)u * kMaxStat * kTile);
-              if (v.y > 0.f) M = fmaxf(M, v.x);
-            }
-            float L = 0.f;
-            for (int u = 0; u < e.n_units; ++u) {
-              const float2 v = __ldcg(parts + (size_t)u * kMaxStat * kTile);
-              if (v.y > 0.f) L += v.y * ex2_approx(v.x - M);
-            }
-            write_row_bias(p, si, g, tok, t % p.G, M + log2f(L));
+            float2 acc = make_float2(-INFINITY, 0.f);
+            for (int u = 0; u < e.n_units; ++u)
+              acc = lse_merge(acc, __ldcg(parts + (size_t)u * kMaxStat * kTile));
+            write_row_bias(p, si, g, tok, t % p.G, acc.x + log2f(acc.y));
           }
         }
       }
-    } else if (e.mode == kModeP2K) {
+    } else {   // kModeP2K
       if (e.n_units == 1) {
 #pragma unroll
         for (int i = 0; i < kMaxStat; ++i) {
           const int key = (e.stat0 + i) * kTile + t;
-          if (i < e.n_stat && key < si.len) p.scores[(size_t)g * p.T + si.start + key] = acc[i];
+          if (i < e.n_stat && key < si.len) p.scores[(size_t)g * p.T + si.start + key] = st[i].y;
         }
       } else {
 #pragma unroll
         for (int i = 0; i < kMaxStat; ++i)
-          if (i < e.n_stat) p.part2[((size_t)unit * kMaxStat + i) * kTile + t] = acc[i];
+          if (i < e.n_stat) p.part2[((size_t)unit * kMaxStat + i) * kTile + t] = st[i].y;
         __threadfence();
-        epi_sync();
+        bar_sync(kBarWG0, 128);
         if (t == 0) *s.last = atomicAdd(&p.c2[ei], 1u) == (uint32_t)(e.n_units - 1);
-        epi_sync();
+        bar_sync(kBarWG0, 128);
         if (*s.last) {
           __threadfence();
           for (int i = 0; i < e.n_stat; ++i) {
@@ -506,11 +521,10 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
       }
     }
   }
-  (void)pass1;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(200)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK, PassArgs p, int pass) {
   using C = Cfg<D>;
@@ -525,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < C::kStages; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
     mbar_init(s.stat_full, 1);
     mbar_init(s.stat_empty, 1);
-    for (int i = 0; i < kTmemBufs; ++i) { mbar_init(&s.tfull[i], 1); mbar_init(&s.tempty[i], kEpiWarps); }
+    for (int i = 0; i < kTmemBufs; ++i) { mbar_init(&s.tfull[i], 1); mbar_init(&s.tempty[i], 4); }
     mbar_init(s.done, 1);
     *s.abort = 0;
     fence_mbar_init();
@@ -555,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mma_issuer<D>(p, s, E, it, tmem);
       __syncwarp();
     } else {
-      epilogue<D>(p, s, E, it, tmem, p1);
+      epilogue<D>(p, s, E, it, tmem);
     }
   }
   tc_fence_before();

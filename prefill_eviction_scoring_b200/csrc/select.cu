@@ -2,30 +2,68 @@
 // the recent window [N-R, N) and the B-R highest scores of [0, N-R), ties to
 // the lower index, reported in ascending order.
 //
-// One CTA per (sequence, KV head).  The (B-R)-th largest score is found by an
-// exact 4-round radix select on the fp32 bit pattern (non-negative floats
-// order like their bits); the kept set is then written in index order with
-// block prefix sums, taking threshold ties lowest index first.
+// One CTA per (sequence, KV head).  Scores are non-negative, so their fp32
+// bit patterns order like the values.  The (B-R)-th largest pattern tau is
+// found exactly by a radix select over 12 + 10 + 10 bits; after the first
+// digit only the candidates that still match the prefix are kept (compacted
+// in shared memory), so later rounds touch few elements.  The kept set is
+// then written in index order with block prefix sums, taking threshold ties
+// lowest index first.  The pool is staged in shared memory when it fits.
 #include "waits_internal.cuh"
 
 namespace waits {
 namespace {
 
 constexpr int kSelThreads = 1024;
+constexpr int kBins1 = 4096;          // first digit: bits 20..31
+constexpr int kBins2 = 1024;          // then bits 10..19 and 0..9
+constexpr int kCand = 8192;           // candidate list capacity (smem)
+constexpr int kCache = 24576;         // pool entries staged in smem (96 KB)
 
 __device__ inline uint32_t order_key(float s) {
   const uint32_t u = __float_as_uint(s);
   return u == 0x80000000u ? 0u : u;   // -0 ranks with +0
 }
 
+// Warp 0 scans `hist[0..nb)` from the top bin down and finds the digit whose
+// bin holds the need-th largest element; returns it (and the count above it)
+// through shared memory.
+__device__ void find_digit(const uint32_t* hist, int nb, int need, uint32_t* s_digit,
+                           int* s_above) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x >= 32) return;
+  const int per = nb / 32;                 // bins per lane, descending
+  const int top = nb - 1 - lane * per;
+  uint32_t tot = 0;
+  for (int i = 0; i < per; ++i) tot += hist[top - i];
+  uint32_t incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint32_t excl = incl - tot;
+  if ((int)excl < need && (int)incl >= need) {
+    uint32_t cum = excl;
+    for (int i = 0; i < per; ++i) {
+      const uint32_t c = hist[top - i];
+      if ((int)(cum + c) >= need) { *s_digit = (uint32_t)(top - i); *s_above = (int)cum; break; }
+      cum += c;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const float* __restrict__ scores, const int32_t* __restrict__ cu, int nseq, int T,
     int Hkv, int R, int B, int32_t* __restrict__ idx, int32_t* __restrict__ kept_len,
     uint32_t* status) {
-  __shared__ uint32_t hist[256];
+  extern __shared__ uint32_t dyn_smem[];
+  uint32_t* cache = dyn_smem;                                  // [kCache] staged keys
+  int* cand = reinterpret_cast<int*>(dyn_smem + kCache);       // [kCand] candidates
+  __shared__ uint32_t hist[kBins1];
   __shared__ int64_t sh[32];
   __shared__ uint32_t s_digit;
-  __shared__ int s_above;
+  __shared__ int s_above, s_ncand;
   const int tid = threadIdx.x;
   const int s = blockIdx.x / Hkv, g = blockIdx.x % Hkv;
   const int lo = cu[s], hi = cu[s + 1];
@@ -48,63 +86,67 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   const int want = B - R;          // positions taken from the pool by score
   const int pool = N - R;
   const float* sc = scores + (size_t)g * T + lo;
-  const int lane = tid & 31, warp = tid >> 5;
+  const bool cached = pool <= kCache;
+  if (cached)
+    for (int k = tid; k < pool; k += blockDim.x) cache[k] = order_key(__ldg(sc + k));
+  auto key = [&](int k) -> uint32_t { return cached ? cache[k] : order_key(__ldg(sc + k)); };
 
-  uint32_t prefix = 0, pmask = 0;
+  uint32_t tau = 0;
   int need = want;
   if (want > 0) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
-      __syncthreads();
-      for (int k = tid; k < pool; k += blockDim.x) {
-        const uint32_t u = order_key(sc[k]);
-        const bool match = (u & pmask) == prefix;
-        const uint32_t dg = (u >> shift) & 255u;
-        const unsigned m = __ballot_sync(__activemask(), match);
-        if (match) {
-          const unsigned peers = __match_any_sync(m, dg);
-          if (lane == __ffs(peers) - 1) atomicAdd(&hist[dg], (uint32_t)__popc(peers));
-        }
+    // ---- digit 1: bits 20..31 over the whole pool
+    for (int i = tid; i < kBins1; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int k = tid; k < pool; k += blockDim.x) atomicAdd(&hist[key(k) >> 20], 1u);
+    __syncthreads();
+    find_digit(hist, kBins1, need, &s_digit, &s_above);
+    __syncthreads();
+    uint32_t prefix = s_digit << 20, pmask = 0xFFF00000u;
+    need -= s_above;
+    // ---- digits 2 and 3 (bits 10..19, 0..9) over the matching candidates
+    if (tid == 0) s_ncand = 0;
+    for (int i = tid; i < kBins2; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int k = tid; k < pool; k += blockDim.x) {
+      const uint32_t u = key(k);
+      if ((u & pmask) == prefix) {
+        const int slot = atomicAdd(&s_ncand, 1);
+        if (slot < kCand) cand[slot] = k;
+        atomicAdd(&hist[(u >> 10) & 1023u], 1u);
       }
-      __syncthreads();
-      if (warp == 0) {
-        // lane L owns bins 255-8L ... 248-8L (descending)
-        uint32_t c[8];
-        uint32_t tot = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { c[i] = hist[255 - 8 * lane - i]; tot += c[i]; }
-        uint32_t incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
+    }
+    __syncthreads();
+    const int ncand = s_ncand;
+    const bool listed = ncand <= kCand;
+    for (int shift = 10; shift >= 0; shift -= 10) {
+      if (shift == 0) {
+        for (int i = tid; i < kBins2; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        const int n = listed ? ncand : pool;
+        for (int q = tid; q < n; q += blockDim.x) {
+          const int k = listed ? cand[q] : q;
+          const uint32_t u = key(k);
+          if ((u & pmask) == prefix) atomicAdd(&hist[u & 1023u], 1u);
         }
-        const uint32_t excl = incl - tot;
-        if ((int)excl < need && (int)incl >= need) {
-          uint32_t cum = excl;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if ((int)(cum + c[i]) >= need) { s_digit = 255 - 8 * lane - i; s_above = (int)cum; break; }
-            cum += c[i];
-          }
-        }
+        __syncthreads();
       }
+      find_digit(hist, kBins2, need, &s_digit, &s_above);
       __syncthreads();
       prefix |= s_digit << shift;
-      pmask |= 255u << shift;
+      pmask |= 1023u << shift;
       need -= s_above;
       __syncthreads();
     }
+    tau = prefix;
   }
-  const uint32_t tau = prefix;
 
-  // ascending output: thread tid owns positions [c0, c1)
+  // ---- ascending output: thread tid owns positions [c0, c1)
   const int per = (N + blockDim.x - 1) / blockDim.x;
   const int c0 = min(N, tid * per), c1 = min(N, c0 + per);
   int n_gt = 0, n_eq = 0;
   if (want > 0) {
     for (int k = c0; k < min(c1, pool); ++k) {
-      const uint32_t u = order_key(sc[k]);
+      const uint32_t u = key(k);
       n_gt += u > tau;
       n_eq += u == tau;
     }
@@ -118,7 +160,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   for (int k = c0; k < c1; ++k) {
     bool keep = k >= pool;
     if (!keep && want > 0) {
-      const uint32_t u = order_key(sc[k]);
+      const uint32_t u = key(k);
       if (u > tau) keep = true;
       else if (u == tau) { keep = eq_seen < take_eq; ++eq_seen; }
     }
@@ -131,8 +173,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int T, int Hkv,
                           int R, int B, int32_t* idx, int32_t* kept_len, uint32_t* status,
                           cudaStream_t s) {
-  select_kernel<<<nseq * Hkv, kSelThreads, 0, s>>>(scores, cu, nseq, T, Hkv, R, B, idx,
-                                                   kept_len, status);
+  const int dyn = (kCache + kCand) * (int)sizeof(uint32_t);
+  cudaError_t err = cudaFuncSetAttribute(select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+  if (err != cudaSuccess) return err;
+  select_kernel<<<nseq * Hkv, kSelThreads, dyn, s>>>(scores, cu, nseq, T, Hkv, R, B, idx,
+                                                     kept_len, status);
   return cudaGetLastError();
 }
 

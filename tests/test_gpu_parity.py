@@ -170,3 +170,25 @@ def test_host_buffer_entry_point():
     kv = 1233 * 2 * 128 * 2 * 2
     q_active = 2 * 120 * 14 * 128 * 2          # ~b + 90/a rows per sequence
     assert kv < hc.h2d_bytes < kv + q_active + 4096   # only the active Q rows
+
+
+@pytest.mark.parametrize("lens,R,B,levels", [
+    ((20000,), 64, 2048, 50),          # pool staged in shared memory
+    ((40000, 3000), 16, 1024, 7),      # pool read from global memory
+    ((50000,), 16, 4096, 1),           # every score equal: candidate list overflows
+    ((9000,), 0, 300, 100000),         # nearly distinct scores, R = 0
+])
+def test_select_exact_on_synthetic_scores(lens, R, B, levels):
+    """waits_select alone, on scores with controlled ties, equals the
+    oracle's selection of the same fp32 values."""
+    from prefill_eviction_scoring_b200 import api
+    g = torch.Generator(device="cuda")
+    g.manual_seed(123)
+    Hkv, T = 3, sum(lens)
+    s = torch.randint(0, levels, (Hkv, T), generator=g, device="cuda").float() / 64.0
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device="cuda")
+    idx, kept = api.select(s, cu, recent_budget=R, budget=B)
+    torch.cuda.synchronize()
+    ref_idx, ref_kept = oracle.select(s.double().cpu().numpy(), cu.cpu().numpy(), R, B)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_array_equal(kept.cpu().numpy(), ref_kept)
