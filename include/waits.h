@@ -78,6 +78,13 @@ int32_t waits_abi_version(void);
 const char* waits_strerror(waits_status status);
 
 /*
+ * Description of the last CUDA runtime failure seen by a call on this host
+ * thread (which step failed and CUDA's error name), "" if none.  The string
+ * is owned by the library and stays valid until the next call that fails.
+ */
+const char* waits_last_error(void);
+
+/*
  * Bytes of device workspace that waits_score / waits_compress need for
  * `shape` (any a, b, R, B).  Host-only; touches no device state.
  * Errors: WAITS_ERR_ARG if shape or bytes is NULL; shape errors as below.

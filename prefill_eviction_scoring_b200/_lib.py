@@ -55,6 +55,7 @@ _PSHAPE = ctypes.POINTER(Shape)
 SIGNATURES = {
     "waits_abi_version": (_I, []),
     "waits_strerror": (ctypes.c_char_p, [_I]),
+    "waits_last_error": (ctypes.c_char_p, []),
     "waits_workspace_size": (_I, [_PSHAPE, ctypes.POINTER(_SZ)]),
     "waits_score": (_I, [_PSHAPE, _P, _P, _F, _I, _P, _P, _SZ, _P]),
     "waits_select": (_I, [_PSHAPE, _P, _I, _I, _P, _P, _P, _SZ, _P]),
@@ -95,5 +96,8 @@ def load(path: str = LIB_PATH):
 
 def check(fn: str, status: int):
     if status != WAITS_OK:
-        msg = load().waits_strerror(status).decode()
+        lib = load()
+        msg = lib.waits_strerror(status).decode()
+        if status == 5:
+            msg += " [" + lib.waits_last_error().decode() + "]"
         raise WaitsError(fn, status, msg)

@@ -524,7 +524,7 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
 }
 
 template <int D>
-__global__ void __maxnreg__(200)
+__global__ void __maxnreg__(192)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK, PassArgs p, int pass) {
   using C = Cfg<D>;

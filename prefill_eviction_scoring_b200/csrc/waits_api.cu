@@ -1,6 +1,7 @@
 // C ABI of libwaits.so: host-side validation, workspace carving and launches
 // on the caller's stream.  Declarations and contracts: include/waits.h.
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 
 #include "waits_internal.cuh"
@@ -8,6 +9,14 @@
 using namespace waits;
 
 namespace {
+
+thread_local char g_last_error[256] = "";
+
+waits_status cuda_fail(const char* what, cudaError_t err) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", what, cudaGetErrorName(err),
+           cudaGetErrorString(err));
+  return WAITS_ERR_CUDA;
+}
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -59,7 +68,7 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   const Layout L = layout_of(s);
   uint8_t* base = static_cast<uint8_t*>(ws);
   const int grid = grid_size();
-  if (grid <= 0) return WAITS_ERR_CUDA;
+  if (grid <= 0) return cuda_fail("device query", cudaGetLastError());
   PlanArgs pa{};
   pa.cu = s->cu_seqlens;
   pa.nseq = s->nseq;
@@ -83,7 +92,8 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   pa.max_u1 = L.max_u1;
   pa.max_u2 = L.max_u2;
   pa.scores = scores;
-  if (launch_plan(pa, st) != cudaSuccess) return WAITS_ERR_CUDA;
+  cudaError_t err = launch_plan(pa, st);
+  if (err != cudaSuccess) return cuda_fail("planner launch", err);
 
   PassArgs p{};
   p.Q = static_cast<const uint16_t*>(Q);
@@ -108,7 +118,8 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   p.part2 = reinterpret_cast<float*>(base + L.part2);
   p.scores = scores;
   p.status = &pa.hdr->status;
-  if (launch_score_passes(p, grid, st) != cudaSuccess) return WAITS_ERR_CUDA;
+  err = launch_score_passes(p, grid, st);
+  if (err != cudaSuccess) return cuda_fail("scorer launch", err);
   return WAITS_OK;
 }
 
@@ -142,6 +153,8 @@ waits_status check_compact_args(const void* K, const void* V, const int32_t* idx
 extern "C" {
 
 int32_t waits_abi_version(void) { return WAITS_ABI_VERSION; }
+
+const char* waits_last_error(void) { return g_last_error; }
 
 const char* waits_strerror(waits_status st) {
   switch (st) {
@@ -181,11 +194,11 @@ waits_status waits_select(const waits_shape* shape, const float* scores, int32_t
   waits_status st = check_shape(shape);
   if (st == WAITS_OK) st = check_select_args(scores, R, B, idx, kept_len);
   if (st != WAITS_OK) return st;
-  if (launch_select(scores, shape->cu_seqlens, shape->nseq, shape->total_tokens,
-                    shape->num_kv_heads, R, B, idx, kept_len,
-                    status_word(workspace, workspace_bytes),
-                    static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return WAITS_ERR_CUDA;
+  const cudaError_t err = launch_select(scores, shape->cu_seqlens, shape->nseq,
+                                        shape->total_tokens, shape->num_kv_heads, R, B, idx,
+                                        kept_len, status_word(workspace, workspace_bytes),
+                                        static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail("select launch", err);
   return WAITS_OK;
 }
 
@@ -195,12 +208,12 @@ waits_status waits_compact(const waits_shape* shape, const void* K, const void* 
   waits_status st = check_shape(shape);
   if (st == WAITS_OK) st = check_compact_args(K, V, idx, kept_len, B, K_out, V_out);
   if (st != WAITS_OK) return st;
-  if (launch_compact(static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
-                     shape->cu_seqlens, idx, kept_len, shape->nseq, shape->num_kv_heads,
-                     shape->head_dim, B, static_cast<uint16_t*>(K_out),
-                     static_cast<uint16_t*>(V_out), status_word(workspace, workspace_bytes),
-                     static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return WAITS_ERR_CUDA;
+  const cudaError_t err = launch_compact(
+      static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V), shape->cu_seqlens, idx,
+      kept_len, shape->nseq, shape->num_kv_heads, shape->head_dim, B,
+      static_cast<uint16_t*>(K_out), static_cast<uint16_t*>(V_out),
+      status_word(workspace, workspace_bytes), static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail("compact launch", err);
   return WAITS_OK;
 }
 
@@ -219,14 +232,14 @@ waits_status waits_compress(const waits_shape* shape, const void* Q, const void*
   st = enqueue_score(shape, Q, K, a, b, scores, workspace, s);
   if (st != WAITS_OK) return st;
   uint32_t* status = status_word(workspace, workspace_bytes);
-  if (launch_select(scores, shape->cu_seqlens, shape->nseq, shape->total_tokens,
-                    shape->num_kv_heads, R, B, idx, kept_len, status, s) != cudaSuccess)
-    return WAITS_ERR_CUDA;
-  if (launch_compact(static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
-                     shape->cu_seqlens, idx, kept_len, shape->nseq, shape->num_kv_heads,
-                     shape->head_dim, B, static_cast<uint16_t*>(K_out),
-                     static_cast<uint16_t*>(V_out), status, s) != cudaSuccess)
-    return WAITS_ERR_CUDA;
+  cudaError_t err = launch_select(scores, shape->cu_seqlens, shape->nseq, shape->total_tokens,
+                                  shape->num_kv_heads, R, B, idx, kept_len, status, s);
+  if (err != cudaSuccess) return cuda_fail("select launch", err);
+  err = launch_compact(static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
+                       shape->cu_seqlens, idx, kept_len, shape->nseq, shape->num_kv_heads,
+                       shape->head_dim, B, static_cast<uint16_t*>(K_out),
+                       static_cast<uint16_t*>(V_out), status, s);
+  if (err != cudaSuccess) return cuda_fail("compact launch", err);
   return WAITS_OK;
 }
 
