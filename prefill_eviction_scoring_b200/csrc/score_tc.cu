@@ -29,7 +29,15 @@ using namespace sm100;
 
 constexpr int kWGs = 2;                              // epilogue warpgroups
 constexpr int kEpiThreads = kWGs * 128;
-constexpr int kThreads = kEpiThreads + 64;           // + producer warp + MMA warp
+constexpr int kThreads = kEpiThreads + 128;          // + producer/MMA warpgroup
+// Register split (setmaxnreg): launched at 168 per thread (3 warps per SM
+// quadrant); the producer/MMA warpgroup drops to 40 and the two epilogue
+// warpgroups rise to 232: 128*40 + 256*232 = 384*168.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsProducer = 40;
+constexpr int kRegsEpilogue = 232;
+static_assert(128 * kRegsProducer + kEpiThreads * kRegsEpilogue <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr int kProducerWarp = kWGs * 4;
 constexpr int kMmaWarp = kProducerWarp + 1;
 constexpr int kTmemBufs = 2 * kWGs;                  // two 128-column buffers per WG
@@ -524,7 +532,7 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
 }
 
 template <int D>
-__global__ void __maxnreg__(192)
+__global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK, PassArgs p, int pass) {
   using C = Cfg<D>;
@@ -561,16 +569,18 @@ __global__ void __maxnreg__(192)
   UnitIter it;
   const bool have = it.init(E, p1 ? H->n_e1 : H->n_e2, p1 ? H->s1 : H->s2,
                             p1 ? H->p1 : H->p2, blockIdx.x);
-  if (have) {
-    if (warp == kProducerWarp) {
+  if (warp >= kProducerWarp) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+    if (have && warp == kProducerWarp) {
       if (lane == 0) producer<D>(&tmQ, &tmK, p, s, E, it);
       __syncwarp();
-    } else if (warp == kMmaWarp) {
+    } else if (have && warp == kMmaWarp) {
       if (lane == 0) mma_issuer<D>(p, s, E, it, tmem);
       __syncwarp();
-    } else {
-      epilogue<D>(p, s, E, it, tmem);
     }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpilogue));
+    if (have) epilogue<D>(p, s, E, it, tmem);
   }
   tc_fence_before();
   __syncthreads();
@@ -624,7 +634,19 @@ cudaError_t launch_d(const PassArgs& a, int grid, cudaStream_t st) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   score_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, a, 1);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if ((err = cudaGetLastError()) != cudaSuccess) {
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, score_tc_kernel<D>);
+    int dev = 0, optin = 0, regs = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaDeviceGetAttribute(&regs, cudaDevAttrMaxRegistersPerBlock, dev);
+    set_error_detail("scorer: regs %d, max threads %d, local %zu B, static smem %zu B, "
+                     "dynamic %zu of opt-in %d B, block regs %d, threads %d",
+                     fa.numRegs, fa.maxThreadsPerBlock, fa.localSizeBytes, fa.sharedSizeBytes,
+                     smem, optin, regs, kThreads);
+    return err;
+  }
   score_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, a, 2);
   return cudaGetLastError();
 }

@@ -6,15 +6,19 @@
 
 #include "waits_internal.cuh"
 
+#include <cstdarg>
+
 using namespace waits;
 
 namespace {
 
-thread_local char g_last_error[256] = "";
+thread_local char g_last_error[512] = "";
+thread_local char g_detail[256] = "";
 
 waits_status cuda_fail(const char* what, cudaError_t err) {
-  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", what, cudaGetErrorName(err),
-           cudaGetErrorString(err));
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)%s%s", what, cudaGetErrorName(err),
+           cudaGetErrorString(err), g_detail[0] ? "; " : "", g_detail);
+  g_detail[0] = 0;
   return WAITS_ERR_CUDA;
 }
 
@@ -149,6 +153,15 @@ waits_status check_compact_args(const void* K, const void* V, const int32_t* idx
 }
 
 }  // namespace
+
+namespace waits {
+void set_error_detail(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+}
+}  // namespace waits
 
 extern "C" {
 

@@ -187,6 +187,9 @@ struct PassArgs {
   uint32_t* status;
 };
 
+// Extra text appended to the next waits_last_error() message (host only).
+void set_error_detail(const char* fmt, ...);
+
 // Host-side launchers (one per translation unit).
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
 cudaError_t launch_score_passes(const PassArgs& a, int grid, cudaStream_t s);
