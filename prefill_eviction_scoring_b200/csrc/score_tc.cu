@@ -400,8 +400,8 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
     const Entry e = E[ei];
     const SeqInfo si = p.seqs[e.seq];
     const int g = e.g;
+    bar_sync(kBarAll, kEpiThreads);   // warpgroup 0 has read the previous unit's states
     for (int i = 0; i < kMaxStat; ++i) { my_m[i * kTile] = -INFINITY; my_l[i * kTile] = 0.f; }
-    bar_sync(kBarAll, kEpiThreads);   // previous unit fully merged
     if (e.mode == kModeP2Q) {
       for (int i = wg; i < e.n_stat; i += kWGs)
         s.bias_stat[i * kTile + t] = qrow_bias(p, si, g, e.stat0 + i, t);
