@@ -274,6 +274,26 @@ struct Cols {
   }
 };
 
+__device__ inline float2 f2(float x, float y) { return make_float2(x, y); }
+__device__ inline float hsum8(const float2 (&a)[4]) {
+  const float2 s = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+  return s.x + s.y;
+}
+
+// sum_c 2^(v_c * sc + off) over all 128 columns, packed fp32x2 arithmetic.
+__device__ inline float exp_sum_full(const Cols& v, float sc, float off) {
+  const float2 sc2 = f2(sc, sc), off2 = f2(off, off);
+  float2 a[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) a[k] = f2(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < kTile; c += 2) {
+    const float2 x = __ffma2_rn(f2(u2f(v.r[c]), u2f(v.r[c + 1])), sc2, off2);
+    a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], f2(ex2_approx(x.x), ex2_approx(x.y)));
+  }
+  return hsum8(a);
+}
+
 // Pass 1, one 128-key tile of this thread's row (keys c < nv are causal):
 // l += sum_c 2^(v_c*scale2 - m), m = first maximum seen, moved up only when
 // the running sum would leave the safe fp32 range.
@@ -285,16 +305,21 @@ __device__ inline void p1_pair(const Cols& v, int nv, float sc, float& m, float&
     for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, c < nv ? u2f(v.r[c]) * sc : -INFINITY);
     m = mx;
   }
-  const float nm = -m;
-  float a[8];
+  float t;
+  if (nv == kTile) {
+    t = exp_sum_full(v, sc, -m);
+  } else {
+    const float nm = -m;
+    float a[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) a[k] = 0.f;
+    for (int k = 0; k < 8; ++k) a[k] = 0.f;
 #pragma unroll
-  for (int c = 0; c < kTile; ++c) {
-    const float x = fmaf(u2f(v.r[c]), sc, nm);
-    a[c & 7] += ex2_approx(c < nv ? x : -INFINITY);
+    for (int c = 0; c < kTile; ++c) {
+      const float x = fmaf(u2f(v.r[c]), sc, nm);
+      a[c & 7] += ex2_approx(c < nv ? x : -INFINITY);
+    }
+    t = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
   }
-  const float t = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
   if (l + t <= kRebaseLimit) {
     l += t;
     return;
@@ -314,12 +339,33 @@ __device__ inline void p1_pair(const Cols& v, int nv, float sc, float& m, float&
 }
 
 // Pass 2, one 128-row Q tile for this thread's key: sum over columns
-// c in [c_lo, ncols) of 2^(v_c*scale2 + bias_c).
+// c in [c_lo, ncols) of 2^(v_c*scale2 + bias_c) (bias is -inf past the rows).
 __device__ inline float p2_pair(const Cols& v, int c_lo, int ncols, float sc, const float* bias) {
+  const float4* b4 = reinterpret_cast<const float4*>(bias);
+  if (c_lo == 0) {
+    const float2 sc2 = f2(sc, sc);
+    float2 a[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) a[k] = f2(0.f, 0.f);
+#pragma unroll
+    for (int cb = 0; cb < kTile; cb += 32) {
+      if (cb < ncols) {
+#pragma unroll
+        for (int c = cb; c < cb + 32; c += 4) {
+          const float4 b = b4[c / 4];
+          const float2 x0 = __ffma2_rn(f2(u2f(v.r[c]), u2f(v.r[c + 1])), sc2, f2(b.x, b.y));
+          const float2 x1 = __ffma2_rn(f2(u2f(v.r[c + 2]), u2f(v.r[c + 3])), sc2, f2(b.z, b.w));
+          a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], f2(ex2_approx(x0.x), ex2_approx(x0.y)));
+          a[((c >> 1) + 1) & 3] =
+              __fadd2_rn(a[((c >> 1) + 1) & 3], f2(ex2_approx(x1.x), ex2_approx(x1.y)));
+        }
+      }
+    }
+    return hsum8(a);
+  }
   float a[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) a[k] = 0.f;
-  const float4* b4 = reinterpret_cast<const float4*>(bias);
 #pragma unroll
   for (int cb = 0; cb < kTile; cb += 32) {
     if (cb < ncols) {

@@ -17,8 +17,9 @@ namespace {
 constexpr int kSelThreads = 1024;
 constexpr int kBins1 = 4096;          // first digit: bits 20..31
 constexpr int kBins2 = 1024;          // then bits 10..19 and 0..9
-constexpr int kCand = 8192;           // candidate list capacity (smem)
-constexpr int kCache = 24576;         // pool entries staged in smem (96 KB)
+constexpr int kCand = 4096;           // candidate list capacity (smem)
+constexpr int kCache = 49152;         // pool entries staged in smem (192 KB)
+constexpr int kBatch = 8;             // loads in flight per thread when streaming
 
 __device__ inline uint32_t order_key(float s) {
   const uint32_t u = __float_as_uint(s);
@@ -87,8 +88,42 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   const int pool = N - R;
   const float* sc = scores + (size_t)g * T + lo;
   const bool cached = pool <= kCache;
-  if (cached)
-    for (int k = tid; k < pool; k += blockDim.x) cache[k] = order_key(__ldg(sc + k));
+  // Visit every pool position k (in no particular order) with its key; keys
+  // come from shared memory when staged, else from global memory with
+  // kBatch independent loads in flight per thread.
+  auto for_each = [&](auto&& f) {
+    const int step = kBatch * (int)blockDim.x;
+    for (int base = tid; base < pool; base += step) {
+      uint32_t u[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int k = base + i * (int)blockDim.x;
+        u[i] = k < pool ? (cached ? cache[k] : order_key(__ldg(sc + k))) : 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int k = base + i * (int)blockDim.x;
+        if (k < pool) f(k, u[i]);
+      }
+    }
+  };
+  if (cached) {
+    const int step = kBatch * (int)blockDim.x;
+    for (int base = tid; base < pool; base += step) {
+      float x[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int k = base + i * (int)blockDim.x;
+        x[i] = k < pool ? __ldg(sc + k) : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int k = base + i * (int)blockDim.x;
+        if (k < pool) cache[k] = order_key(x[i]);
+      }
+    }
+    __syncthreads();
+  }
   auto key = [&](int k) -> uint32_t { return cached ? cache[k] : order_key(__ldg(sc + k)); };
 
   uint32_t tau = 0;
@@ -97,7 +132,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     // ---- digit 1: bits 20..31 over the whole pool
     for (int i = tid; i < kBins1; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    for (int k = tid; k < pool; k += blockDim.x) atomicAdd(&hist[key(k) >> 20], 1u);
+    for_each([&](int, uint32_t u) { atomicAdd(&hist[u >> 20], 1u); });
     __syncthreads();
     find_digit(hist, kBins1, need, &s_digit, &s_above);
     __syncthreads();
@@ -107,14 +142,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     if (tid == 0) s_ncand = 0;
     for (int i = tid; i < kBins2; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    for (int k = tid; k < pool; k += blockDim.x) {
-      const uint32_t u = key(k);
+    for_each([&](int k, uint32_t u) {
       if ((u & pmask) == prefix) {
         const int slot = atomicAdd(&s_ncand, 1);
         if (slot < kCand) cand[slot] = k;
         atomicAdd(&hist[(u >> 10) & 1023u], 1u);
       }
-    }
+    });
     __syncthreads();
     const int ncand = s_ncand;
     const bool listed = ncand <= kCand;
@@ -122,11 +156,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
       if (shift == 0) {
         for (int i = tid; i < kBins2; i += blockDim.x) hist[i] = 0;
         __syncthreads();
-        const int n = listed ? ncand : pool;
-        for (int q = tid; q < n; q += blockDim.x) {
-          const int k = listed ? cand[q] : q;
-          const uint32_t u = key(k);
-          if ((u & pmask) == prefix) atomicAdd(&hist[u & 1023u], 1u);
+        if (listed) {
+          for (int q = tid; q < ncand; q += blockDim.x) {
+            const uint32_t u = key(cand[q]);
+            if ((u & pmask) == prefix) atomicAdd(&hist[u & 1023u], 1u);
+          }
+        } else {
+          for_each([&](int, uint32_t u) {
+            if ((u & pmask) == prefix) atomicAdd(&hist[u & 1023u], 1u);
+          });
         }
         __syncthreads();
       }
