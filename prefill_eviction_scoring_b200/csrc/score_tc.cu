@@ -31,11 +31,11 @@ constexpr int kWGs = 2;                              // epilogue warpgroups
 constexpr int kEpiThreads = kWGs * 128;
 constexpr int kThreads = kEpiThreads + 128;          // + producer/MMA warpgroup
 // Register split (setmaxnreg): launched at 168 per thread (3 warps per SM
-// quadrant); the producer/MMA warpgroup drops to 40 and the two epilogue
-// warpgroups rise to 232: 128*40 + 256*232 = 384*168.
+// quadrant); the producer/MMA warpgroup drops to 56 and the two epilogue
+// warpgroups rise to 224: 128*56 + 256*224 = 384*168.
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsProducer = 40;
-constexpr int kRegsEpilogue = 232;
+constexpr int kRegsProducer = 56;
+constexpr int kRegsEpilogue = 224;
 static_assert(128 * kRegsProducer + kEpiThreads * kRegsEpilogue <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr int kProducerWarp = kWGs * 4;
@@ -180,9 +180,9 @@ out:
 }
 
 // ---------------------------------------------------------- MMA issuer ---
-// Streamed tiles are taken two at a time; the pairs of the first go to
-// epilogue warpgroup 0, those of the second to warpgroup 1, interleaved so
-// both groups always have work.  Each group owns two TMEM buffers.
+// Pairs of stationary slot i go to epilogue warpgroup i % 2, so both groups
+// work on the same streamed tile and the next one is prefetched meanwhile.
+// Each group owns two TMEM buffers.
 template <int D>
 __device__ void mma_issuer(const PassArgs& p, const Smem& s, const Entry* E, UnitIter it,
                            uint32_t tmem) {
@@ -199,44 +199,37 @@ __device__ void mma_issuer(const PassArgs& p, const Smem& s, const Entry* E, Uni
     if (!mbar_wait(s.stat_full, uph, s.abort, p.status, kWaitLimitNs)) goto out;
     uph ^= 1u;
     tc_fence_after();
-    const int n = st1 - st0;
-    for (int ls = 0; ls < n; ls += kWGs) {
-      const int nw = n - ls < kWGs ? n - ls : kWGs;     // streamed tiles this round
-      int stg[kWGs];
-      for (int w = 0; w < nw; ++w) {
-        stg[w] = stage;
-        if (!mbar_wait(&s.full[stage], sph, s.abort, p.status, kWaitLimitNs)) goto out;
-        if (++stage == C::kStages) { stage = 0; sph ^= 1u; }
-      }
+    for (int st = st0; st < st1; ++st) {
+      const int o = e.step0 + st;
+      if (!mbar_wait(&s.full[stage], sph, s.abort, p.status, kWaitLimitNs)) goto out;
       tc_fence_after();
+      const uint32_t sa = strm0 + stage * C::kTileBytes;
       for (int i = 0; i < e.n_stat; ++i) {
-        for (int w = 0; w < nw; ++w) {
-          const int o = e.step0 + st0 + ls + w;
-          int j, kt;
-          pair_tiles(e, o, i, j, kt);
-          if (!pair_live(si, j, kt, p.tokq)) continue;
-          const int buf = 2 * w + (int)(kpair[w] & 1u);
-          const uint32_t ph = (kpair[w] >> 1) & 1u;
-          if (!mbar_wait(&s.tempty[buf], ph ^ 1u, s.abort, p.status, kWaitLimitNs)) goto out;
-          tc_fence_after();
-          const uint32_t sa = strm0 + stg[w] * C::kTileBytes;
-          const uint32_t ta = stat0 + i * C::kTileBytes;
-          // P1: A = Q (stationary), B = K (streamed); P2Q: A = K (streamed),
-          // B = Q (stationary); P2K: A = K (stationary), B = Q (streamed).
-          const uint32_t a_base = e.mode == kModeP2Q ? sa : ta;
-          const uint32_t b_base = e.mode == kModeP2Q ? ta : sa;
-          const uint32_t d_tmem = tmem + (uint32_t)(buf * kTile);
+        int j, kt;
+        pair_tiles(e, o, i, j, kt);
+        if (!pair_live(si, j, kt, p.tokq)) continue;
+        const int w = i & 1;
+        const int buf = 2 * w + (int)(kpair[w] & 1u);
+        const uint32_t ph = (kpair[w] >> 1) & 1u;
+        if (!mbar_wait(&s.tempty[buf], ph ^ 1u, s.abort, p.status, kWaitLimitNs)) goto out;
+        tc_fence_after();
+        const uint32_t ta = stat0 + i * C::kTileBytes;
+        // P1: A = Q (stationary), B = K (streamed); P2Q: A = K (streamed),
+        // B = Q (stationary); P2K: A = K (stationary), B = Q (streamed).
+        const uint32_t a_base = e.mode == kModeP2Q ? sa : ta;
+        const uint32_t b_base = e.mode == kModeP2Q ? ta : sa;
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * kTile);
 #pragma unroll
-          for (int k = 0; k < C::kKSteps; ++k) {
-            const uint32_t off = (uint32_t)((k >> 2) * C::kSubBytes + (k & 3) * 32);
-            mma_bf16(d_tmem, sdesc_kmajor_sw128(a_base + off),
-                     sdesc_kmajor_sw128(b_base + off), idesc, k > 0 ? 1u : 0u);
-          }
-          mma_commit(&s.tfull[buf]);
-          ++kpair[w];
+        for (int k = 0; k < C::kKSteps; ++k) {
+          const uint32_t off = (uint32_t)((k >> 2) * C::kSubBytes + (k & 3) * 32);
+          mma_bf16(d_tmem, sdesc_kmajor_sw128(a_base + off), sdesc_kmajor_sw128(b_base + off),
+                   idesc, k > 0 ? 1u : 0u);
         }
+        mma_commit(&s.tfull[buf]);
+        ++kpair[w];
       }
-      for (int w = 0; w < nw; ++w) mma_commit(&s.empty[stg[w]]);
+      mma_commit(&s.empty[stage]);
+      if (++stage == C::kStages) { stage = 0; sph ^= 1u; }
     }
     mma_commit(s.stat_empty);
   }
@@ -431,39 +424,39 @@ template <int D>
 __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitIter it,
                          uint32_t tmem) {
   const int tid = threadIdx.x;               // 0..255
-  const int wg = tid >> 7;                    // warpgroup
+  const int wg = tid >> 7;                    // warpgroup: owns stationary slots wg, wg + 2
   const int t = tid & 127;                    // TMEM lane == row (pass 1) / key (pass 2)
   const int lane = tid & 31;
   const uint32_t lane_addr = tmem + ((uint32_t)((t >> 5) * 32) << 16);
-  const int bar_wg = kBarWG0 + wg;
-  float* my_m = s.st_m + wg * kMaxStat * kTile + t;
-  float* my_l = s.st_l + wg * kMaxStat * kTile + t;
   uint32_t kp = 0;          // pairs consumed by this warpgroup
-  int sstep = 0;            // streamed steps consumed by this warpgroup
+  int sstep = 0;            // streamed steps seen (double-buffered shared data)
   bool ok = true;           // false after a timeout: keep every barrier, skip the work
   int ei, st0, st1, unit;
   while (it.next(ei, st0, st1, unit)) {
     const Entry e = E[ei];
     const SeqInfo si = p.seqs[e.seq];
     const int g = e.g;
-    bar_sync(kBarAll, kEpiThreads);   // warpgroup 0 has read the previous unit's states
-    for (int i = 0; i < kMaxStat; ++i) { my_m[i * kTile] = -INFINITY; my_l[i * kTile] = 0.f; }
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};   // P1 row state / P2K sums
+    bar_sync(kBarAll, kEpiThreads);   // the previous unit's shared data is no longer read
     if (e.mode == kModeP2Q) {
       for (int i = wg; i < e.n_stat; i += kWGs)
         s.bias_stat[i * kTile + t] = qrow_bias(p, si, g, e.stat0 + i, t);
       bar_sync(kBarAll, kEpiThreads);
     }
-    const int n = st1 - st0;
-    for (int ls = wg; ls < n; ls += kWGs) {
-      const int o = e.step0 + st0 + ls;
-      float* bias_o = s.bias_strm + (wg * 2 + (sstep & 1)) * kTile;
+    for (int st = st0; st < st1; ++st) {
+      const int o = e.step0 + st;
+      const int sb = sstep & 1;
       ++sstep;
+      float* bias_o = s.bias_strm + sb * kTile;
       if (e.mode == kModeP2K) {
-        bias_o[t] = qrow_bias(p, si, g, o, t);
-        bar_sync(bar_wg, 128);
+        if (wg == 0) bias_o[t] = qrow_bias(p, si, g, o, t);
+        bar_sync(kBarAll, kEpiThreads);
       }
       float col = 0.f;
-      for (int i = 0; i < e.n_stat; ++i) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int i = wg + 2 * k;
+        if (i >= e.n_stat) break;
         int j, kt;
         pair_tiles(e, o, i, j, kt);
         if (!pair_live(si, j, kt, p.tokq)) continue;
@@ -484,10 +477,7 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
           const bool row_ok = t < p.tokq * p.G && tok < si.len;
           int nv = row_ok ? tok - kt * kTile + 1 : 0;
           nv = nv > kTile ? kTile : nv;
-          float m = my_m[i * kTile], l = my_l[i * kTile];
-          p1_pair(v, nv, p.scale2, m, l);
-          my_m[i * kTile] = m;
-          my_l[i * kTile] = l;
+          p1_pair(v, nv, p.scale2, m[k], l[k]);
         } else {
           const int key = kt * kTile + t;
           const int f = si.q0 + j * p.tokq;
@@ -495,83 +485,72 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
           const int ncols = min(p.tokq, si.len - f) * p.G;   // valid columns (uniform)
           const float* bias = e.mode == kModeP2K ? bias_o : s.bias_stat + i * kTile;
           const float a2 = p2_pair(v, c_lo, ncols, p.scale2, bias);
-          if (e.mode == kModeP2K) my_l[i * kTile] += a2; else col += a2;
+          if (e.mode == kModeP2K) l[k] += a2; else col += a2;
         }
       }
-      if (e.mode == kModeP2Q && ok) {
-        const int key = o * kTile + t;
-        if (key < si.len) p.scores[(size_t)g * p.T + si.start + key] = col;
+      if (e.mode == kModeP2Q) {
+        // the two warpgroups' halves of this key's column sum
+        float* part = s.st_l + (sb * kWGs + wg) * kTile;
+        part[t] = col;
+        bar_sync(kBarAll, kEpiThreads);
+        if (wg == 0 && ok) {
+          const int key = o * kTile + t;
+          if (key < si.len)
+            p.scores[(size_t)g * p.T + si.start + key] = part[t] + part[kTile + t];
+        }
       }
     }
 
-    // ---- unit results: both warpgroups' partial states are merged by WG 0
+    // ---- unit results: each warpgroup writes the slots it owns
     const bool fail = bar_vote_or(kBarAll, kEpiThreads, !ok || *s.abort);
-    float2 st[kMaxStat];
-    if (!fail && wg == 0 && e.mode != kModeP2Q) {
-#pragma unroll
-      for (int i = 0; i < kMaxStat; ++i) {
-        const float2 a = make_float2(my_m[i * kTile], my_l[i * kTile]);
-        const float2 b = make_float2(my_m[kMaxStat * kTile + i * kTile],
-                                     my_l[kMaxStat * kTile + i * kTile]);
-        st[i] = e.mode == kModeP1 ? lse_merge(a, b) : make_float2(0.f, a.y + b.y);
-      }
-    }
     if (fail) { ok = false; continue; }
-    if (wg != 0 || e.mode == kModeP2Q) continue;
-    if (e.mode == kModeP1) {
-      if (e.n_units == 1) {
+    if (e.mode == kModeP2Q) continue;
+    const bool p1 = e.mode == kModeP1;
+    if (e.n_units == 1) {
 #pragma unroll
-        for (int i = 0; i < kMaxStat; ++i) {
+      for (int k = 0; k < 2; ++k) {
+        const int i = wg + 2 * k;
+        if (i >= e.n_stat) break;
+        if (p1) {
           const int tok = si.q0 + (e.stat0 + i) * p.tokq + t / p.G;
-          if (i < e.n_stat && t < p.tokq * p.G && tok < si.len)
-            write_row_bias(p, si, g, tok, t % p.G, st[i].x + log2f(st[i].y));
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < kMaxStat; ++i)
-          if (i < e.n_stat) p.part1[((size_t)unit * kMaxStat + i) * kTile + t] = st[i];
-        __threadfence();
-        bar_sync(kBarWG0, 128);
-        if (t == 0) *s.last = atomicAdd(&p.c1[ei], 1u) == (uint32_t)(e.n_units - 1);
-        bar_sync(kBarWG0, 128);
-        if (*s.last) {
-          __threadfence();
-          for (int i = 0; i < e.n_stat; ++i) {
-            const int tok = si.q0 + (e.stat0 + i) * p.tokq + t / p.G;
-            if (t >= p.tokq * p.G || tok >= si.len) continue;
-            const float2* parts = p.part1 + ((size_t)e.unit_base * kMaxStat + i) * kTile + t;
-            float2 acc = make_float2(-INFINITY, 0.f);
-            for (int u = 0; u < e.n_units; ++u)
-              acc = lse_merge(acc, __ldcg(parts + (size_t)u * kMaxStat * kTile));
-            write_row_bias(p, si, g, tok, t % p.G, acc.x + log2f(acc.y));
-          }
+          if (t < p.tokq * p.G && tok < si.len)
+            write_row_bias(p, si, g, tok, t % p.G, m[k] + log2f(l[k]));
+        } else {
+          const int key = (e.stat0 + i) * kTile + t;
+          if (key < si.len) p.scores[(size_t)g * p.T + si.start + key] = l[k];
         }
       }
-    } else {   // kModeP2K
-      if (e.n_units == 1) {
+      continue;
+    }
 #pragma unroll
-        for (int i = 0; i < kMaxStat; ++i) {
-          const int key = (e.stat0 + i) * kTile + t;
-          if (i < e.n_stat && key < si.len) p.scores[(size_t)g * p.T + si.start + key] = st[i].y;
-        }
+    for (int k = 0; k < 2; ++k) {
+      const int i = wg + 2 * k;
+      if (i >= e.n_stat) break;
+      const size_t slot = ((size_t)unit * kMaxStat + i) * kTile + t;
+      if (p1) p.part1[slot] = make_float2(m[k], l[k]); else p.part2[slot] = l[k];
+    }
+    __threadfence();
+    bar_sync(kBarAll, kEpiThreads);
+    if (tid == 0)
+      *s.last = atomicAdd(p1 ? &p.c1[ei] : &p.c2[ei], 1u) == (uint32_t)(e.n_units - 1);
+    bar_sync(kBarAll, kEpiThreads);
+    if (!*s.last) continue;
+    __threadfence();
+    for (int i = wg; i < e.n_stat; i += kWGs) {
+      const size_t base = ((size_t)e.unit_base * kMaxStat + i) * kTile + t;
+      if (p1) {
+        const int tok = si.q0 + (e.stat0 + i) * p.tokq + t / p.G;
+        if (t >= p.tokq * p.G || tok >= si.len) continue;
+        float2 acc = make_float2(-INFINITY, 0.f);
+        for (int u = 0; u < e.n_units; ++u)
+          acc = lse_merge(acc, __ldcg(p.part1 + base + (size_t)u * kMaxStat * kTile));
+        write_row_bias(p, si, g, tok, t % p.G, acc.x + log2f(acc.y));
       } else {
-#pragma unroll
-        for (int i = 0; i < kMaxStat; ++i)
-          if (i < e.n_stat) p.part2[((size_t)unit * kMaxStat + i) * kTile + t] = st[i].y;
-        __threadfence();
-        bar_sync(kBarWG0, 128);
-        if (t == 0) *s.last = atomicAdd(&p.c2[ei], 1u) == (uint32_t)(e.n_units - 1);
-        bar_sync(kBarWG0, 128);
-        if (*s.last) {
-          __threadfence();
-          for (int i = 0; i < e.n_stat; ++i) {
-            const int key = (e.stat0 + i) * kTile + t;
-            float sum = 0.f;
-            for (int u = 0; u < e.n_units; ++u)
-              sum += __ldcg(p.part2 + ((size_t)(e.unit_base + u) * kMaxStat + i) * kTile + t);
-            if (key < si.len) p.scores[(size_t)g * p.T + si.start + key] = sum;
-          }
-        }
+        const int key = (e.stat0 + i) * kTile + t;
+        float sum = 0.f;
+        for (int u = 0; u < e.n_units; ++u)
+          sum += __ldcg(p.part2 + base + (size_t)u * kMaxStat * kTile);
+        if (key < si.len) p.scores[(size_t)g * p.T + si.start + key] = sum;
       }
     }
   }
