@@ -273,7 +273,33 @@ __device__ inline float hsum8(const float2 (&a)[4]) {
   return s.x + s.y;
 }
 
-// sum_c 2^(v_c * sc + off) over all 128 columns, packed fp32x2 arithmetic.
+// Columns of every 32 whose exponential runs on the FMA pipe instead of the
+// MUFU (which does 16 ex2 per clock per SM and bounds the unmasked passes).
+constexpr int kPolyPer32 = 10;
+
+// 2^x for a pair of fp32 values on the FMA/ALU pipes (Cody-Waite split plus
+// a polynomial): x = n + f with n = rint(x) and f in [-1/2, 1/2], 2^f by a
+// degree-3 minimax polynomial for relative error (max 7.5e-5; coefficients
+// fitted by a Remez exchange), 2^n added to the exponent bits.  x is clamped
+// to [-125, 127] so the result stays a normal fp32 number.
+__device__ inline float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.0f;              // 1.5 * 2^23: rint via fadd
+  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261113f, c3 = 0.05517167f;
+  x = f2(fminf(fmaxf(x.x, -125.f), 127.f), fminf(fmaxf(x.y, -125.f), 127.f));
+  const float2 t = __fadd2_rn(x, f2(kMagic, kMagic));
+  const float2 n = __fadd2_rn(t, f2(-kMagic, -kMagic));
+  const float2 fr = __ffma2_rn(n, f2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(f2(c3, c3), fr, f2(c2, c2));
+  q = __ffma2_rn(q, fr, f2(c1, c1));
+  q = __ffma2_rn(q, fr, f2(c0, c0));
+  // the magic's low 9 bits are zero, so (bits(t) << 23) == n << 23
+  const int ex = __float_as_int(t.x) << 23, ey = __float_as_int(t.y) << 23;
+  return f2(__int_as_float(__float_as_int(q.x) + ex), __int_as_float(__float_as_int(q.y) + ey));
+}
+
+// sum_c 2^(v_c * sc + off) over all 128 columns, packed fp32x2 arithmetic;
+// of every 32 columns the first 32 - kPolyPer32 use the MUFU, the rest the
+// polynomial.
 __device__ inline float exp_sum_full(const Cols& v, float sc, float off) {
   const float2 sc2 = f2(sc, sc), off2 = f2(off, off);
   float2 a[4];
@@ -282,7 +308,9 @@ __device__ inline float exp_sum_full(const Cols& v, float sc, float off) {
 #pragma unroll
   for (int c = 0; c < kTile; c += 2) {
     const float2 x = __ffma2_rn(f2(u2f(v.r[c]), u2f(v.r[c + 1])), sc2, off2);
-    a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], f2(ex2_approx(x.x), ex2_approx(x.y)));
+    const float2 e = ((c & 31) < 32 - kPolyPer32) ? f2(ex2_approx(x.x), ex2_approx(x.y))
+                                                   : exp2_poly2(x);
+    a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], e);
   }
   return hsum8(a);
 }
@@ -348,9 +376,13 @@ __device__ inline float p2_pair(const Cols& v, int c_lo, int ncols, float sc, co
           const float4 b = b4[c / 4];
           const float2 x0 = __ffma2_rn(f2(u2f(v.r[c]), u2f(v.r[c + 1])), sc2, f2(b.x, b.y));
           const float2 x1 = __ffma2_rn(f2(u2f(v.r[c + 2]), u2f(v.r[c + 3])), sc2, f2(b.z, b.w));
-          a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], f2(ex2_approx(x0.x), ex2_approx(x0.y)));
-          a[((c >> 1) + 1) & 3] =
-              __fadd2_rn(a[((c >> 1) + 1) & 3], f2(ex2_approx(x1.x), ex2_approx(x1.y)));
+          const float2 e0 = ((c & 31) < 32 - kPolyPer32) ? f2(ex2_approx(x0.x), ex2_approx(x0.y))
+                                                          : exp2_poly2(x0);
+          const float2 e1 = (((c + 2) & 31) < 32 - kPolyPer32)
+                                ? f2(ex2_approx(x1.x), ex2_approx(x1.y))
+                                : exp2_poly2(x1);
+          a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], e0);
+          a[((c >> 1) + 1) & 3] = __fadd2_rn(a[((c >> 1) + 1) & 3], e1);
         }
       }
     }

@@ -26,6 +26,30 @@ __device__ inline uint32_t order_key(float s) {
   return u == 0x80000000u ? 0u : u;   // -0 ranks with +0
 }
 
+// Histogram add from every active lane: lanes holding the same bin are
+// merged first, so a warp issues one shared-memory atomic per distinct bin
+// (scores cluster in a few bins; unmerged atomics would serialise).
+__device__ inline void hist_add(uint32_t* hist, uint32_t bin) {
+  const unsigned peers = __match_any_sync(__activemask(), bin);
+  if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+}
+
+// Append k to the candidate list with one atomic per warp.
+__device__ inline void cand_push(int* cand, int* count, bool take, int k) {
+  const unsigned act = __activemask();
+  const unsigned m = __ballot_sync(act, take);
+  if (!m) return;
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(m) - 1;
+  int base = 0;
+  if (lane == leader) base = atomicAdd(count, __popc(m));
+  base = __shfl_sync(act, base, leader);
+  if (take) {
+    const int slot = base + __popc(m & ((1u << lane) - 1u));
+    if (slot < kCand) cand[slot] = k;
+  }
+}
+
 // Warp 0 scans `hist[0..nb)` from the top bin down and finds the digit whose
 // bin holds the need-th largest element; returns it (and the count above it)
 // through shared memory.
@@ -132,7 +156,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     // ---- digit 1: bits 20..31 over the whole pool
     for (int i = tid; i < kBins1; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    for_each([&](int, uint32_t u) { atomicAdd(&hist[u >> 20], 1u); });
+    for_each([&](int, uint32_t u) { hist_add(hist, u >> 20); });
     __syncthreads();
     find_digit(hist, kBins1, need, &s_digit, &s_above);
     __syncthreads();
@@ -143,11 +167,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     for (int i = tid; i < kBins2; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     for_each([&](int k, uint32_t u) {
-      if ((u & pmask) == prefix) {
-        const int slot = atomicAdd(&s_ncand, 1);
-        if (slot < kCand) cand[slot] = k;
-        atomicAdd(&hist[(u >> 10) & 1023u], 1u);
-      }
+      const bool take = (u & pmask) == prefix;
+      cand_push(cand, &s_ncand, take, k);
+      if (take) hist_add(hist, (u >> 10) & 1023u);
     });
     __syncthreads();
     const int ncand = s_ncand;
@@ -159,11 +181,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
         if (listed) {
           for (int q = tid; q < ncand; q += blockDim.x) {
             const uint32_t u = key(cand[q]);
-            if ((u & pmask) == prefix) atomicAdd(&hist[u & 1023u], 1u);
+            if ((u & pmask) == prefix) hist_add(hist, u & 1023u);
           }
         } else {
           for_each([&](int, uint32_t u) {
-            if ((u & pmask) == prefix) atomicAdd(&hist[u & 1023u], 1u);
+            if ((u & pmask) == prefix) hist_add(hist, u & 1023u);
           });
         }
         __syncthreads();

@@ -15,7 +15,7 @@ namespace waits {
 constexpr int kTile = 128;      // keys per K tile; max packed rows per Q tile
 constexpr int kMaxStat = 4;     // stationary tiles held by one work unit
 constexpr int kMaxGrid = 1024;  // upper bound on persistent CTAs (sizing)
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 256;
 
 // A Q tile packs `tokq` consecutive query positions x G heads of one KV
 // group: packed row r <-> position q0 + j*tokq + r / G, head g*G + r % G.
@@ -122,7 +122,7 @@ __device__ inline int first_active_row(int N, float a, int b) {
 }
 
 // --------------------------------------------------------- block scans ---
-// Exclusive prefix sum over a block of kPlanThreads threads.
+// Exclusive prefix sum over the threads of a block (a multiple of 32, <= 1024).
 __device__ inline int64_t block_exclusive_scan(int64_t v, int64_t* total, int64_t* sh /*[32]*/) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int64_t x = v;
