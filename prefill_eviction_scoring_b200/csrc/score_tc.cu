@@ -278,20 +278,22 @@ __device__ inline float hsum8(const float2 (&a)[4]) {
 constexpr int kPolyPer32 = 10;
 
 // 2^x for a pair of fp32 values on the FMA/ALU pipes (Cody-Waite split plus
-// a polynomial): x = n + f with n = rint(x) and f in [-1/2, 1/2], 2^f by a
-// degree-3 minimax polynomial for relative error (max 7.5e-5; coefficients
-// fitted by a Remez exchange), 2^n added to the exponent bits.  x is clamped
-// to [-125, 127] so the result stays a normal fp32 number.
+// a polynomial): x = n + f with n = rint(x) and f in [-1/2, 1/2];
+// 2^f ~ 1 + f (c1 + f (c2 + f c3)), the relative-error minimax cubic with the
+// constant term held at 1 (max relative error 1.0e-4; fitted by linear
+// programming on a dense grid), so integer x gives exact powers of two; 2^n
+// is added to the exponent bits.  x is clamped to [-125, 127] so the result
+// stays a normal fp32 number.
 __device__ inline float2 exp2_poly2(float2 x) {
   constexpr float kMagic = 12582912.0f;              // 1.5 * 2^23: rint via fadd
-  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261113f, c3 = 0.05517167f;
+  constexpr float c1 = 0.69328290f, c2 = 0.24221097f, c3 = 0.05500906f;
   x = f2(fminf(fmaxf(x.x, -125.f), 127.f), fminf(fmaxf(x.y, -125.f), 127.f));
   const float2 t = __fadd2_rn(x, f2(kMagic, kMagic));
   const float2 n = __fadd2_rn(t, f2(-kMagic, -kMagic));
   const float2 fr = __ffma2_rn(n, f2(-1.f, -1.f), x);
   float2 q = __ffma2_rn(f2(c3, c3), fr, f2(c2, c2));
   q = __ffma2_rn(q, fr, f2(c1, c1));
-  q = __ffma2_rn(q, fr, f2(c0, c0));
+  q = __ffma2_rn(q, fr, f2(1.f, 1.f));
   // the magic's low 9 bits are zero, so (bits(t) << 23) == n << 23
   const int ex = __float_as_int(t.x) << 23, ey = __float_as_int(t.y) << 23;
   return f2(__int_as_float(__float_as_int(q.x) + ex), __int_as_float(__float_as_int(q.y) + ey));
