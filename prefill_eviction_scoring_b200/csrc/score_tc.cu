@@ -273,9 +273,12 @@ __device__ inline float hsum8(const float2 (&a)[4]) {
   return s.x + s.y;
 }
 
-// Columns of every 32 whose exponential runs on the FMA pipe instead of the
-// MUFU (which does 16 ex2 per clock per SM and bounds the unmasked passes).
-constexpr int kPolyPer32 = 10;
+// Column pairs whose exponential runs on the FMA pipe instead of the MUFU
+// (which does 16 ex2 per clock per SM and bounds the unmasked passes): bit
+// (pair index mod 8) of this mask.  Two in eight, spread out, measured best;
+// more makes the warps issue-bound.
+constexpr uint32_t kPolyPairs = 0x88u;
+__device__ constexpr bool poly_col(int c) { return (kPolyPairs >> ((c >> 1) & 7)) & 1u; }
 
 // 2^x for a pair of fp32 values on the FMA/ALU pipes (Cody-Waite split plus
 // a polynomial): x = n + f with n = rint(x) and f in [-1/2, 1/2];
@@ -300,8 +303,7 @@ __device__ inline float2 exp2_poly2(float2 x) {
 }
 
 // sum_c 2^(v_c * sc + off) over all 128 columns, packed fp32x2 arithmetic;
-// of every 32 columns the first 32 - kPolyPer32 use the MUFU, the rest the
-// polynomial.
+// the column pairs picked by kPolyPairs use the polynomial, the rest the MUFU.
 __device__ inline float exp_sum_full(const Cols& v, float sc, float off) {
   const float2 sc2 = f2(sc, sc), off2 = f2(off, off);
   float2 a[4];
@@ -310,8 +312,7 @@ __device__ inline float exp_sum_full(const Cols& v, float sc, float off) {
 #pragma unroll
   for (int c = 0; c < kTile; c += 2) {
     const float2 x = __ffma2_rn(f2(u2f(v.r[c]), u2f(v.r[c + 1])), sc2, off2);
-    const float2 e = ((c & 31) < 32 - kPolyPer32) ? f2(ex2_approx(x.x), ex2_approx(x.y))
-                                                   : exp2_poly2(x);
+    const float2 e = poly_col(c) ? exp2_poly2(x) : f2(ex2_approx(x.x), ex2_approx(x.y));
     a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], e);
   }
   return hsum8(a);
@@ -378,11 +379,9 @@ __device__ inline float p2_pair(const Cols& v, int c_lo, int ncols, float sc, co
           const float4 b = b4[c / 4];
           const float2 x0 = __ffma2_rn(f2(u2f(v.r[c]), u2f(v.r[c + 1])), sc2, f2(b.x, b.y));
           const float2 x1 = __ffma2_rn(f2(u2f(v.r[c + 2]), u2f(v.r[c + 3])), sc2, f2(b.z, b.w));
-          const float2 e0 = ((c & 31) < 32 - kPolyPer32) ? f2(ex2_approx(x0.x), ex2_approx(x0.y))
-                                                          : exp2_poly2(x0);
-          const float2 e1 = (((c + 2) & 31) < 32 - kPolyPer32)
-                                ? f2(ex2_approx(x1.x), ex2_approx(x1.y))
-                                : exp2_poly2(x1);
+          const float2 e0 = poly_col(c) ? exp2_poly2(x0) : f2(ex2_approx(x0.x), ex2_approx(x0.y));
+          const float2 e1 =
+              poly_col(c + 2) ? exp2_poly2(x1) : f2(ex2_approx(x1.x), ex2_approx(x1.y));
           a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], e0);
           a[((c >> 1) + 1) & 3] = __fadd2_rn(a[((c >> 1) + 1) & 3], e1);
         }

@@ -18,7 +18,11 @@ constexpr int kSelThreads = 1024;
 constexpr int kBins1 = 4096;          // first digit: bits 20..31
 constexpr int kBins2 = 1024;          // then bits 10..19 and 0..9
 constexpr int kCand = 4096;           // candidate list capacity (smem)
-constexpr int kCache = 49152;         // pool entries staged in smem (192 KB)
+constexpr int kCache = 45056;         // pool entries staged in smem (~176 KB)
+// Staged key k lives at k + k/32: one pad word per 32 keeps both the
+// strided visits and the per-thread contiguous output scan conflict-free.
+__device__ inline int cpos(int k) { return k + (k >> 5); }
+constexpr int kCacheWords = kCache + kCache / 32;
 constexpr int kBatch = 8;             // loads in flight per thread when streaming
 
 __device__ inline uint32_t order_key(float s) {
@@ -83,8 +87,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     int Hkv, int R, int B, int32_t* __restrict__ idx, int32_t* __restrict__ kept_len,
     uint32_t* status) {
   extern __shared__ uint32_t dyn_smem[];
-  uint32_t* cache = dyn_smem;                                  // [kCache] staged keys
-  int* cand = reinterpret_cast<int*>(dyn_smem + kCache);       // [kCand] candidates
+  uint32_t* cache = dyn_smem;                                  // staged keys (padded)
+  int* cand = reinterpret_cast<int*>(dyn_smem + kCacheWords);  // [kCand] candidates
   __shared__ uint32_t hist[kBins1];
   __shared__ int64_t sh[32];
   __shared__ uint32_t s_digit;
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 #pragma unroll
       for (int i = 0; i < kBatch; ++i) {
         const int k = base + i * (int)blockDim.x;
-        u[i] = k < pool ? (cached ? cache[k] : order_key(__ldg(sc + k))) : 0u;
+        u[i] = k < pool ? (cached ? cache[cpos(k)] : order_key(__ldg(sc + k))) : 0u;
       }
 #pragma unroll
       for (int i = 0; i < kBatch; ++i) {
@@ -143,12 +147,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 #pragma unroll
       for (int i = 0; i < kBatch; ++i) {
         const int k = base + i * (int)blockDim.x;
-        if (k < pool) cache[k] = order_key(x[i]);
+        if (k < pool) cache[cpos(k)] = order_key(x[i]);
       }
     }
     __syncthreads();
   }
-  auto key = [&](int k) -> uint32_t { return cached ? cache[k] : order_key(__ldg(sc + k)); };
+  auto key = [&](int k) -> uint32_t {
+    return cached ? cache[cpos(k)] : order_key(__ldg(sc + k));
+  };
 
   uint32_t tau = 0;
   int need = want;
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int T, int Hkv,
                           int R, int B, int32_t* idx, int32_t* kept_len, uint32_t* status,
                           cudaStream_t s) {
-  const int dyn = (kCache + kCand) * (int)sizeof(uint32_t);
+  const int dyn = (kCacheWords + kCand) * (int)sizeof(uint32_t);
   cudaError_t err = cudaFuncSetAttribute(select_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
   if (err != cudaSuccess) return err;
