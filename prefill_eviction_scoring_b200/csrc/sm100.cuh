@@ -52,6 +52,20 @@ __device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Same, but the thread may be suspended in hardware for up to `hint_ns`
+// while the phase is incomplete, instead of spinning on the issue port that
+// it shares with the math warps of its SM sub-partition.
+__device__ inline bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 
 // Wait for the phase with `parity` to complete.  Gives up after `limit_ns`
 // (or at once when *abort is set by another role), flags `status` and
@@ -61,8 +75,8 @@ __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* a
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 63u) == 0) {
+    if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
+    if ((n & 7u) == 0) {
       if (*abort) return false;
       if (globaltimer() - t0 > limit_ns) {
         *abort = 1;
