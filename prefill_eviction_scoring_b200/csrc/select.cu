@@ -82,6 +82,148 @@ __device__ void find_digit(const uint32_t* hist, int nb, int need, uint32_t* s_d
   }
 }
 
+// ------------------------------------------------------------ fast path ---
+// Pools of up to kSelThreads * kPer keys: every thread holds a contiguous run
+// of kPer keys in registers.  A sorted sample of one key per thread brackets
+// the (want)-th largest key; one pass counts the keys above the bracket and
+// collects those inside it (value, index); a bitonic sort of the collected
+// keys (value descending, index ascending) gives the exact threshold and how
+// many of its ties are taken.  Returns false (nothing written) when the
+// bracket misses or overflows, and the caller runs the radix path.
+constexpr int kPer = 32;
+constexpr int kFastCand = 2048;
+
+__device__ inline void bitonic_desc_u32(uint32_t* a, int n) {
+  for (int k = 2; k <= n; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int ij = i ^ j;
+        if (ij > i) {
+          const uint32_t x = a[i], y = a[ij];
+          if (((i & k) == 0) == (x < y)) { a[i] = y; a[ij] = x; }
+        }
+      }
+    }
+  __syncthreads();
+}
+
+__device__ inline void bitonic_desc_u64(uint64_t* a, int n) {
+  for (int k = 2; k <= n; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int ij = i ^ j;
+        if (ij > i) {
+          const uint64_t x = a[i], y = a[ij];
+          if (((i & k) == 0) == (x < y)) { a[i] = y; a[ij] = x; }
+        }
+      }
+    }
+  __syncthreads();
+}
+
+__device__ bool select_fast(const float* __restrict__ sc, int pool, int N, int want, int B,
+                            int32_t* __restrict__ out, uint32_t* smem, int64_t* sh,
+                            int* s_ncand) {
+  __shared__ uint32_t s_tau;
+  __shared__ int s_need, s_ok;
+  const int tid = threadIdx.x;
+  const int base = tid * kPer;
+  uint32_t u[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) u[j] = base + j < pool ? order_key(__ldg(sc + base + j)) : 0u;
+  int64_t tot;
+  uint32_t tau = 0;
+  int need = want;
+  if (want > 0) {
+    // sample: the first key of every thread's run (runs past the pool: 0)
+    uint32_t* samp = smem;
+    const int S = (pool + kPer - 1) / kPer;
+    samp[tid] = base < pool ? u[0] : 0u;
+    bitonic_desc_u32(samp, kSelThreads);
+    const double p = (double)want / pool;
+    const int r = (int)((double)want * S / pool);
+    const int delta = (int)ceilf(4.0f * sqrtf((float)(S * p * (1.0 - p)))) + 4;
+    const int hr = r - delta, lr = r + delta;
+    const uint32_t t_hi = hr >= 0 ? samp[hr] : 0xFFFFFFFFu;
+    const uint32_t t_lo = lr < S ? samp[lr] : 0u;
+    __syncthreads();
+    // count keys above the bracket, collect those inside it
+    uint64_t* cand = reinterpret_cast<uint64_t*>(smem + kSelThreads);
+    if (tid == 0) *s_ncand = 0;
+    __syncthreads();
+    int above = 0;
+    const int lane = tid & 31;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const bool valid = base + j < pool;
+      above += valid && u[j] > t_hi;
+      const bool take = valid && u[j] <= t_hi && u[j] >= t_lo;
+      const unsigned m = __ballot_sync(0xffffffffu, take);
+      int slot0 = 0;
+      if (m) {
+        if (lane == __ffs(m) - 1) slot0 = atomicAdd(s_ncand, __popc(m));
+        slot0 = __shfl_sync(0xffffffffu, slot0, __ffs(m) - 1);
+        if (take) {
+          const int slot = slot0 + __popc(m & ((1u << lane) - 1u));
+          if (slot < kFastCand)
+            cand[slot] = ((uint64_t)u[j] << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)(base + j));
+        }
+      }
+    }
+    const int n_above = (int)block_exclusive_scan(above, &tot, sh);
+    (void)n_above;
+    const int ab = (int)tot;
+    const int nc = *s_ncand;
+    const bool ok = nc <= kFastCand && ab < want && ab + nc >= want;
+    if (!ok) return false;    // uniform: every thread saw the same totals
+    int n2 = 1;
+    while (n2 < nc) n2 <<= 1;
+    for (int i = nc + tid; i < n2; i += blockDim.x) cand[i] = 0ull;
+    bitonic_desc_u64(cand, n2);
+    if (tid == 0) {
+      const int k = want - ab - 1;                 // the threshold key's place
+      const uint32_t t = (uint32_t)(cand[k] >> 32);
+      int first = k;
+      while (first > 0 && (uint32_t)(cand[first - 1] >> 32) == t) --first;
+      s_tau = t;
+      s_need = (want - ab) - first;                // ties of t that are kept
+    }
+    __syncthreads();
+    tau = s_tau;
+    need = s_need;
+  }
+  // ascending output from the register runs
+  int n_gt = 0, n_eq = 0;
+  if (want > 0) {
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const bool valid = base + j < pool;
+      n_gt += valid && u[j] > tau;
+      n_eq += valid && u[j] == tau;
+    }
+  }
+  const int c0 = min(N, base), c1 = min(N, base + kPer);
+  const int eq_before = (int)block_exclusive_scan(n_eq, &tot, sh);
+  const int take_eq = max(0, min(n_eq, need - eq_before));
+  const int n_rec = max(0, c1 - max(c0, pool));
+  int pos = (int)block_exclusive_scan(n_gt + take_eq + n_rec, &tot, sh);
+  int eq_seen = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int k = base + j;
+    if (k >= N) break;
+    bool keep = k >= pool;
+    if (!keep && want > 0) {
+      if (u[j] > tau) keep = true;
+      else if (u[j] == tau) { keep = eq_seen < take_eq; ++eq_seen; }
+    }
+    if (keep && pos < B) out[pos++] = k;
+  }
+  return true;
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const float* __restrict__ scores, const int32_t* __restrict__ cu, int nseq, int T,
     int Hkv, int R, int B, int32_t* __restrict__ idx, int32_t* __restrict__ kept_len,
@@ -115,6 +257,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   const int want = B - R;          // positions taken from the pool by score
   const int pool = N - R;
   const float* sc = scores + (size_t)g * T + lo;
+  if (N <= kSelThreads * kPer &&
+      select_fast(sc, pool, N, want, B, out, dyn_smem, sh, &s_ncand))
+    return;
   const bool cached = pool <= kCache;
   // Visit every pool position k (in no particular order) with its key; keys
   // come from shared memory when staged, else from global memory with

@@ -107,16 +107,28 @@ __device__ inline float curve_weight(int q, int N, float a, int b) {
 }
 
 // First row whose fp32 weight is non-zero (N if none).  For a > 0 the weight
-// is non-decreasing in q, so a binary search finds it; a = 0 weights every
-// row by 1/2.
+// is non-decreasing in q and vanishes once -a (q - c) passes ~88.7 (expf
+// overflows), so the search starts from that estimate and walks to the
+// exact boundary, falling back to bisection if the walk is long; a = 0
+// weights every row by 1/2.
 __device__ inline int first_active_row(int N, float a, int b) {
   if (N <= 0) return 0;
   if (a == 0.0f) return 0;
-  if (!(curve_weight(N - 1, N, a, b) != 0.0f)) return N;
+  auto active = [&](int q) { return curve_weight(q, N, a, b) != 0.0f; };
+  if (!active(N - 1)) return N;
+  const float c = (float)N - (float)b - 0.5f;
+  float est = ceilf(c - 88.72284f / a);
+  int q = est < 0.f ? 0 : (est > (float)(N - 1) ? N - 1 : (int)est);
+  for (int step = 0; step < 8; ++step) {
+    const bool on = active(q);
+    if (on && (q == 0 || !active(q - 1))) return q;
+    q += on ? -1 : 1;
+    if (q < 0 || q > N - 1) break;
+  }
   int lo = 0, hi = N - 1;
   while (lo < hi) {
     const int mid = lo + (hi - lo) / 2;
-    if (curve_weight(mid, N, a, b) != 0.0f) hi = mid; else lo = mid + 1;
+    if (active(mid)) hi = mid; else lo = mid + 1;
   }
   return lo;
 }
