@@ -40,12 +40,17 @@ UNIT = "tokens/s"
 CONFIG = "llama8b"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1590.0}
 KERNELS_PER_LAYER = 5   # plan, pass 1, pass 2, select, compact
+# DRAM bytes (read + write) of one waits_score call on one llama8b layer, from
+# the ncu capture summarised in profiles/score_tc_select_llama8b_1layer.md
+# (both scorer passes).  Valid only for the scorer source it was taken on.
+PROFILED_SCORER = {"sha256_prefix": "c3b5937b8244de16", "dram_bytes": 68_129_792 + 866_304 +
+                   68_149_760 + 797_696}
 
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--budget", type=int, default=2048)
@@ -88,6 +93,16 @@ def select_compact_bytes(lens, Hkv, d, B):
     rows = sum(min(B, N) for N in lens) * Hkv
     comp = 2 * 2 * rows * d * 2 + len(lens) * Hkv * B * 4
     return sel, comp
+
+
+def profiled_traffic():
+    """ncu DRAM bytes of the scorer, or None when score_tc.cu has changed
+    since the capture."""
+    import hashlib
+    src = os.path.join(ROOT, "prefill_eviction_scoring_b200", "csrc", "score_tc.cu")
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    return PROFILED_SCORER["dram_bytes"] if h.startswith(PROFILED_SCORER["sha256_prefix"]) else None
 
 
 def peaks():
@@ -153,7 +168,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -329,7 +344,7 @@ def run_ours(args):
     achieved_t = flops / (t_score / 1e3) / 1e12
     roof = {"kernel": "scorer (waits_score: planner + pass 1 + pass 2)",
             "bound": "tensor", "achieved": round(achieved_t, 2), "peak": peak_t,
-            "unit": "TFLOP/s", "frac": round(achieved_t / peak_t, 4), "traffic": None,
+            "unit": "TFLOP/s", "frac": round(achieved_t / peak_t, 4), "traffic": profiled_traffic(),
             "peak_kind": f"bf16_tflops_sustained ({pk_kind})",
             "flops_per_launch": flops, "launch_ms": round(t_score, 4)}
     hbm = float(pk.get("hbm_gbs"))
