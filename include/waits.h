@@ -191,6 +191,37 @@ waits_status waits_compress_host(const waits_shape* shape,
                                  size_t* d2h_bytes);
 
 /*
+ * Largest scratch waits_score_static can use: 32 MiB, enough for one
+ * Llama-3.1-8B-shaped layer (N = 32768, 32/8 heads) whose
+ * waits_workspace_size() is 19.2 MiB.
+ */
+#define WAITS_STATIC_WORKSPACE_BYTES (32u << 20)
+
+/*
+ * waits_score without a caller-supplied workspace.  The WAITS pages have no
+ * counterpart of this call: it exists for callers that cannot allocate
+ * device memory -- a plugin whose host engine owns the whole device pool, or
+ * code running where an allocation is forbidden or would synchronise the
+ * device.  The scorer's scratch lives in one file-scope device array of
+ * WAITS_STATIC_WORKSPACE_BYTES that every GPU loading the library keeps
+ * until the process exits; the call allocates nothing.
+ *   Arguments, layouts and results as waits_score.
+ *   Errors: as waits_score; WAITS_ERR_WORKSPACE when
+ *   waits_workspace_size(shape) exceeds WAITS_STATIC_WORKSPACE_BYTES (nothing
+ *   is launched).
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   Every call on a device shares the one array, which keeps the previous
+ *   call's contents; each call rewrites all of it before use.  Calls whose
+ *   work overlaps on the GPU (other streams, other host threads) race on it:
+ *   serialise them.  The device status word of this call lives in the array
+ *   and is not readable through waits_read_device_status.
+ */
+waits_status waits_score_static(const waits_shape* shape, const void* Q, const void* K,
+                                float a, int32_t b, float* scores, void* stream);
+
+/*
  * Synchronise `stream` and read the device status word of `workspace`
  * (bits WAITS_DEV_*; 0 = clean).  The word is cleared at the start of every
  * waits_score / waits_compress.  Errors: ARG, WORKSPACE, CUDA.

@@ -68,7 +68,10 @@ SIGNATURES = {
                                  ctypes.POINTER(_SZ)]),
     "waits_read_device_status": (_I, [_P, _SZ, _P,
                                       ctypes.POINTER(ctypes.c_uint32)]),
+    "waits_score_static": (_I, [_PSHAPE, _P, _P, _F, _I, _P, _P]),
 }
+
+STATIC_WORKSPACE_BYTES = 32 << 20   # WAITS_STATIC_WORKSPACE_BYTES
 
 _lib = None
 

@@ -126,6 +126,31 @@ def score(Q: torch.Tensor, K: torch.Tensor, cu_seqlens: torch.Tensor, *,
     return c.score(Q, K, sigmoid_a, window)
 
 
+def score_static(Q: torch.Tensor, K: torch.Tensor, cu_seqlens: torch.Tensor, *,
+                 sigmoid_a: float, window: int, max_seqlen: Optional[int] = None,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """``waits_score_static``: the scores of :func:`score` with the library's
+    own static scratch instead of a workspace, for callers that must not
+    allocate device memory (pass ``out``, fp32 ``[Hkv, T]``, to allocate
+    nothing here either).  Shapes whose workspace would exceed
+    ``_lib.STATIC_WORKSPACE_BYTES`` are rejected; calls that overlap on the
+    GPU share the scratch and must be serialised."""
+    _need_cuda("Q", Q, torch.bfloat16)
+    _need_cuda("K", K, torch.bfloat16)
+    _need_cuda("cu_seqlens", cu_seqlens, torch.int32)
+    T, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    if out is None:
+        out = torch.empty((Hkv, T), dtype=torch.float32, device=Q.device)
+    _need_cuda("out", out, torch.float32)
+    lib = _lib.load()
+    shape = make_shape(cu_seqlens, T, _max_seqlen(cu_seqlens, max_seqlen), Hq, Hkv, d)
+    st = lib.waits_score_static(ctypes.byref(shape), _ptr(Q), _ptr(K), float(sigmoid_a),
+                                int(window), _ptr(out), _stream(Q.device))
+    _lib.check("waits_score_static", st)
+    return out
+
+
 def select(scores: torch.Tensor, cu_seqlens: torch.Tensor, *, recent_budget: int,
            budget: int, max_seqlen: Optional[int] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """``(idx [nseq, Hkv, B] int32, kept_len [nseq] int32)`` (``waits_select``)."""
