@@ -172,13 +172,16 @@ def test_host_buffer_entry_point():
     assert kv < hc.h2d_bytes < kv + q_active + 4096   # only the active Q rows
 
 
-@pytest.mark.parametrize("lens,R,B,levels", [
-    ((20000,), 64, 2048, 50),          # pool staged in shared memory
-    ((40000, 3000), 16, 1024, 7),      # pool read from global memory
-    ((50000,), 16, 4096, 1),           # every score equal: candidate list overflows
-    ((9000,), 0, 300, 100000),         # nearly distinct scores, R = 0
+@pytest.mark.parametrize("lens,R,B,levels,signed", [
+    ((20000,), 64, 2048, 50, False),          # few levels: many ties at the threshold
+    ((40000, 3000), 16, 1024, 7, False),      # ragged batch
+    ((50000,), 16, 4096, 1, False),           # every score equal
+    ((9000,), 0, 300, 100000, False),         # nearly distinct scores, R = 0
+    ((150000, 700), 16, 2048, 3000, False),   # pool larger than the cluster's shared memory
+    ((5000, 2600), 8, 512, 40, True),         # negative values, -0 and +0
+    ((3000,), 16, 2999, 5, False),            # one pool position dropped
 ])
-def test_select_exact_on_synthetic_scores(lens, R, B, levels):
+def test_select_exact_on_synthetic_scores(lens, R, B, levels, signed):
     """waits_select alone, on scores with controlled ties, equals the
     oracle's selection of the same fp32 values."""
     from prefill_eviction_scoring_b200 import api
@@ -186,6 +189,10 @@ def test_select_exact_on_synthetic_scores(lens, R, B, levels):
     g.manual_seed(123)
     Hkv, T = 3, sum(lens)
     s = torch.randint(0, levels, (Hkv, T), generator=g, device="cuda").float() / 64.0
+    if signed:
+        s = s - (levels // 2) / 64.0
+        s[s == 0] = torch.where(torch.rand(int((s == 0).sum()), generator=g, device="cuda") < 0.5,
+                                -0.0, 0.0)
     cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device="cuda")
     idx, kept = api.select(s, cu, recent_budget=R, budget=B)
     torch.cuda.synchronize()
