@@ -12,6 +12,8 @@ __global__ void __launch_bounds__(256) compact_kernel(
     const int32_t* __restrict__ idx, const int32_t* __restrict__ kept_len, int nseq, int Hkv,
     int chunks /* d / 8 */, int B, uint4* __restrict__ Ko, uint4* __restrict__ Vo,
     uint32_t* status) {
+  pdl_allow_next();
+  pdl_wait();
   const int64_t total = (int64_t)nseq * Hkv * B * chunks;
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
        v += (int64_t)gridDim.x * blockDim.x) {
@@ -52,10 +54,10 @@ cudaError_t launch_compact(const uint16_t* K, const uint16_t* V, const int32_t* 
   const int64_t cap = (int64_t)sms * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  compact_kernel<<<(int)blocks, 256, 0, s>>>(
-      reinterpret_cast<const uint4*>(K), reinterpret_cast<const uint4*>(V), cu, idx, kept_len,
-      nseq, Hkv, d / 8, B, reinterpret_cast<uint4*>(Ko), reinterpret_cast<uint4*>(Vo), status);
-  return cudaGetLastError();
+  return launch_pdl(compact_kernel, dim3((unsigned)blocks), dim3(256), 0, s,
+                    reinterpret_cast<const uint4*>(K), reinterpret_cast<const uint4*>(V), cu,
+                    idx, kept_len, nseq, Hkv, d / 8, B, reinterpret_cast<uint4*>(Ko),
+                    reinterpret_cast<uint4*>(Vo), status);
 }
 
 }  // namespace waits

@@ -139,6 +139,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs p) {
   __shared__ SeqInfo s_seqs[kSmemSeqs];
   const int tid = threadIdx.x;
   if (tid == 0) s_bad = 0;
+  pdl_allow_next();
+  pdl_wait();
   __syncthreads();
   Seqs S{p.nseq <= kSmemSeqs ? s_seqs : nullptr, p.seqs};
 
@@ -219,8 +221,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs p) {
 }  // namespace
 
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s) {
-  plan_kernel<<<1, kPlanThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, a);
 }
 
 }  // namespace waits

@@ -571,18 +571,34 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
     __threadfence();
     for (int i = wg; i < e.n_stat; i += kWGs) {
       const size_t base = ((size_t)e.unit_base * kMaxStat + i) * kTile + t;
+      // the partials of all units, in unit order, eight loads in flight
+      constexpr size_t kStride = (size_t)kMaxStat * kTile;
+      constexpr int kBatch = 8;
       if (p1) {
         const int tok = si.q0 + (e.stat0 + i) * p.tokq + t / p.G;
         if (t >= p.tokq * p.G || tok >= si.len) continue;
         float2 acc = make_float2(-INFINITY, 0.f);
-        for (int u = 0; u < e.n_units; ++u)
-          acc = lse_merge(acc, __ldcg(p.part1 + base + (size_t)u * kMaxStat * kTile));
+        for (int u0 = 0; u0 < e.n_units; u0 += kBatch) {
+          float2 x[kBatch];
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b)
+            x[b] = u0 + b < e.n_units ? __ldcg(p.part1 + base + (size_t)(u0 + b) * kStride)
+                                      : make_float2(-INFINITY, 0.f);
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) acc = lse_merge(acc, x[b]);
+        }
         write_row_bias(p, si, g, tok, t % p.G, acc.x + log2f(acc.y));
       } else {
         const int key = (e.stat0 + i) * kTile + t;
         float sum = 0.f;
-        for (int u = 0; u < e.n_units; ++u)
-          sum += __ldcg(p.part2 + base + (size_t)u * kMaxStat * kTile);
+        for (int u0 = 0; u0 < e.n_units; u0 += kBatch) {
+          float x[kBatch];
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b)
+            x[b] = u0 + b < e.n_units ? __ldcg(p.part2 + base + (size_t)(u0 + b) * kStride) : 0.f;
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) sum += x[b];
+        }
         if (key < si.len) p.scores[(size_t)g * p.T + si.start + key] = sum;
       }
     }
@@ -619,10 +635,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_proxy_async_smem();
   if (warp == kMmaWarp) tmem_alloc(s.tmem_slot, kTmemCols);
   if (warp == kProducerWarp && lane == 0) { prefetch_tensormap(&tmQ); prefetch_tensormap(&tmK); }
+  pdl_allow_next();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s.tmem_slot;
+  pdl_wait();   // the plan (and Q, K) written by earlier kernels are visible from here
 
   UnitIter it;
   const bool have = it.init(E, p1 ? H->n_e1 : H->n_e2, p1 ? H->s1 : H->s2,
@@ -691,8 +709,8 @@ cudaError_t launch_d(const PassArgs& a, int grid, cudaStream_t st) {
   cudaError_t err = cudaFuncSetAttribute(score_tc_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  score_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, a, 1);
-  if ((err = cudaGetLastError()) != cudaSuccess) {
+  if ((err = launch_pdl(score_tc_kernel<D>, dim3(grid), dim3(kThreads), smem, st, mq, mk, a, 1)) !=
+      cudaSuccess) {
     cudaFuncAttributes fa{};
     cudaFuncGetAttributes(&fa, score_tc_kernel<D>);
     int dev = 0, optin = 0, regs = 0;
@@ -705,8 +723,7 @@ cudaError_t launch_d(const PassArgs& a, int grid, cudaStream_t st) {
                      smem, optin, regs, kThreads);
     return err;
   }
-  score_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, a, 2);
-  return cudaGetLastError();
+  return launch_pdl(score_tc_kernel<D>, dim3(grid), dim3(kThreads), smem, st, mq, mk, a, 2);
 }
 
 }  // namespace

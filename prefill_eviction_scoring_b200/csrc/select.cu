@@ -114,6 +114,8 @@ __global__ void __cluster_dims__(kCta, 1, 1) __launch_bounds__(kSelThreads) sele
   __shared__ SelSmem sm;
   cg::cluster_group cl = cg::this_cluster();
   const int tid = threadIdx.x;
+  pdl_allow_next();
+  pdl_wait();
   const int r = (int)cl.block_rank();
   const int sg = blockIdx.x / kCta;
   const int s = sg / Hkv, g = sg % Hkv;
@@ -249,9 +251,8 @@ cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int 
   if (err != cudaSuccess) return err;
   const int64_t grid = (int64_t)nseq * Hkv * kCta;
   if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  select_kernel<<<(unsigned)grid, kSelThreads, dyn, s>>>(scores, cu, nseq, T, Hkv, R, B, idx,
-                                                         kept_len, status);
-  return cudaGetLastError();
+  return launch_pdl(select_kernel, dim3((unsigned)grid), dim3(kSelThreads), (size_t)dyn, s,
+                    scores, cu, nseq, T, Hkv, R, B, idx, kept_len, status);
 }
 
 }  // namespace waits

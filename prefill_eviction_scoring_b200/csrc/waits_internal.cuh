@@ -5,6 +5,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 
 #include "waits.h"
@@ -198,6 +199,34 @@ struct PassArgs {
   float* scores;       // [Hkv, T]
   uint32_t* status;
 };
+
+// ------------------------------------------- programmatic dependent launch ---
+// Every kernel of the path is launched with programmatic stream
+// serialisation: it may start while the previous kernel on the stream is
+// still running, does only its private set-up (shared memory, barriers,
+// tensor memory), then waits for the previous grid to complete and its
+// memory to be visible before it touches global memory.  It lets the next
+// kernel start launching at once; that kernel waits the same way.
+__device__ inline void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ inline void pdl_allow_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Extra text appended to the next waits_last_error() message (host only).
 void set_error_detail(const char* fmt, ...);
