@@ -88,10 +88,14 @@ __device__ Entry make_entry(const Seqs& S, int nseq, int tokq, int i) {
 
 // Fill, scan and split the entries of one pass over the CTAs; entries are
 // regenerated from the sequence table in each sweep rather than re-read.
+// When every entry can have at least one CTA of its own (CTA boundaries at
+// the rounded positions C_e * P / S of the entries' first steps, every entry
+// with at least as many steps as CTAs), each entry gets its own CTAs
+// ("aligned"); otherwise CTAs split the global step range.
 template <bool P1>
 __device__ void plan_pass(const Seqs& S, int nseq, int tokq, int n, int grid, Entry* out,
                           uint32_t* counters, int64_t max_units, int64_t* sh, int64_t* steps,
-                          int* units, int* ctas, bool* overflow) {
+                          int* units, int* ctas, int* aligned_out, bool* overflow) {
   int64_t carry = 0;
   for (int base = 0; base < n; base += blockDim.x) {
     const int i = base + threadIdx.x;
@@ -102,6 +106,25 @@ __device__ void plan_pass(const Seqs& S, int nseq, int tokq, int n, int grid, En
   }
   const int64_t Stot = carry;
   const int64_t P = Stot < (int64_t)grid ? Stot : (int64_t)grid;
+  auto cta_at = [&](int64_t c) { return (c * P + Stot / 2) / Stot; };
+  // can every entry own whole CTAs?
+  bool aligned = n <= P && Stot > 0;
+  {
+    int64_t sb = 0;
+    int bad = 0;
+    for (int base = 0; base < n && aligned; base += blockDim.x) {
+      const int i = base + threadIdx.x;
+      const int64_t v = i < n ? (int64_t)make_entry<P1>(S, nseq, tokq, i).n_steps : 0;
+      int64_t tot;
+      const int64_t c = sb + block_exclusive_scan(v, &tot, sh);
+      sb += tot;
+      if (i < n) {
+        const int64_t nu = cta_at(c + v) - cta_at(c);
+        if (nu < 1 || nu > v) bad = 1;
+      }
+      if (__syncthreads_or(bad)) aligned = false;
+    }
+  }
   int64_t sb = 0, ub = 0;
   for (int base = 0; base < n; base += blockDim.x) {
     const int i = base + threadIdx.x;
@@ -113,14 +136,19 @@ __device__ void plan_pass(const Seqs& S, int nseq, int tokq, int n, int grid, En
     sb += tot;
     int64_t nu = 0;
     if (i < n) {
-      const int64_t f = e.sbase * P / Stot;
-      const int64_t l = (e.sbase + e.n_steps - 1) * P / Stot;
-      e.first_cta = (int)f;
-      nu = l - f + 1;
+      if (aligned) {
+        e.first_cta = (int)cta_at(e.sbase);
+        nu = cta_at(e.sbase + e.n_steps) - e.first_cta;
+      } else {
+        const int64_t f = e.sbase * P / Stot;
+        const int64_t l = (e.sbase + e.n_steps - 1) * P / Stot;
+        e.first_cta = (int)f;
+        nu = l - f + 1;
+      }
       e.n_units = (int)nu;
     }
     const int64_t ux = block_exclusive_scan(nu, &tot, sh);
-    e.unit_base = (int)(ub + ux);
+    e.unit_base = aligned ? e.first_cta : (int)(ub + ux);   // aligned: unit = CTA
     ub += tot;
     if (i < n) {
       out[i] = e;
@@ -130,6 +158,7 @@ __device__ void plan_pass(const Seqs& S, int nseq, int tokq, int n, int grid, En
   *steps = Stot;
   *units = (int)ub;
   *ctas = (int)P;
+  *aligned_out = aligned ? 1 : 0;
   if (ub > max_units) *overflow = true;
 }
 
@@ -182,17 +211,18 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs p) {
       H->status = WAITS_DEV_BAD_SEQLENS;
       H->n_e1 = H->n_e2 = H->n_u1 = H->n_u2 = H->p1 = H->p2 = 0;
       H->s1 = H->s2 = 0;
+      H->aligned1 = H->aligned2 = 0;
     }
     return;
   }
   bool overflow = c1 > p.max_e1 || c2 > p.max_e2;
   int64_t S1 = 0, S2 = 0;
-  int U1 = 0, U2 = 0, P1 = 0, P2 = 0;
+  int U1 = 0, U2 = 0, P1 = 0, P2 = 0, A1 = 0, A2 = 0;
   if (!overflow) {
     plan_pass<true>(S, p.nseq, p.tokq, (int)c1, p.grid, p.e1, p.c1, p.max_u1, sh, &S1, &U1,
-                    &P1, &overflow);
+                    &P1, &A1, &overflow);
     plan_pass<false>(S, p.nseq, p.tokq, (int)c2, p.grid, p.e2, p.c2, p.max_u2, sh, &S2, &U2,
-                     &P2, &overflow);
+                     &P2, &A2, &overflow);
   }
   if (tid == 0) {
     H->status = overflow ? WAITS_DEV_PLAN_OVERFLOW : 0u;
@@ -204,6 +234,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs p) {
     H->p2 = overflow ? 0 : P2;
     H->s1 = S1;
     H->s2 = S2;
+    H->aligned1 = A1;
+    H->aligned2 = A2;
   }
 
   // 2) sequences without any active row score 0 everywhere.
@@ -221,7 +253,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs p) {
 }  // namespace
 
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s) {
-  return launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, a);
+  // few sequences: one warp plans alone (shuffle scans, no block barriers)
+  const int threads = a.nseq <= 64 ? 32 : kPlanThreads;
+  return launch_pdl(plan_kernel, dim3(1), dim3(threads), 0, s, a);
 }
 
 }  // namespace waits

@@ -322,6 +322,9 @@ __device__ inline float exp_sum_full(const Cols& v, float sc, float off) {
 // l += sum_c 2^(v_c*scale2 - m), m = first maximum seen, moved up only when
 // the running sum would leave the safe fp32 range.
 __device__ inline void p1_pair(const Cols& v, int nv, float sc, float& m, float& l) {
+  // one path per warp: a warp whose rows are not all fully causal (or absent)
+  // takes the masked path, which also serves its full rows
+  const bool full_warp = __all_sync(0xffffffffu, nv == kTile || nv <= 0);
   if (nv <= 0) return;
   if (m == -INFINITY) {
     float mx = -INFINITY;
@@ -330,7 +333,7 @@ __device__ inline void p1_pair(const Cols& v, int nv, float sc, float& m, float&
     m = mx;
   }
   float t;
-  if (nv == kTile) {
+  if (full_warp) {
     t = exp_sum_full(v, sc, -m);
   } else {
     const float nm = -m;
@@ -366,7 +369,7 @@ __device__ inline void p1_pair(const Cols& v, int nv, float sc, float& m, float&
 // c in [c_lo, ncols) of 2^(v_c*scale2 + bias_c) (bias is -inf past the rows).
 __device__ inline float p2_pair(const Cols& v, int c_lo, int ncols, float sc, const float* bias) {
   const float4* b4 = reinterpret_cast<const float4*>(bias);
-  if (c_lo == 0) {
+  if (__all_sync(0xffffffffu, c_lo == 0)) {   // one path per warp
     const float2 sc2 = f2(sc, sc);
     float2 a[4];
 #pragma unroll
@@ -569,37 +572,60 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
     bar_sync(kBarAll, kEpiThreads);
     if (!*s.last) continue;
     __threadfence();
-    for (int i = wg; i < e.n_stat; i += kWGs) {
-      const size_t base = ((size_t)e.unit_base * kMaxStat + i) * kTile + t;
-      // the partials of all units, in unit order, eight loads in flight
-      constexpr size_t kStride = (size_t)kMaxStat * kTile;
-      constexpr int kBatch = 8;
-      if (p1) {
+    // each thread merges row t of the slots wg and wg + 2: the partials of all
+    // units, in unit order, up to 40 loads in flight
+    constexpr size_t kStride = (size_t)kMaxStat * kTile;
+    constexpr int kBatch = 20;
+    const int nu = e.n_units;
+    if (p1) {
+      float2 acc[2] = {make_float2(-INFINITY, 0.f), make_float2(-INFINITY, 0.f)};
+      for (int u0 = 0; u0 < nu; u0 += kBatch) {
+        float2 x[2][kBatch];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int i = wg + 2 * k;
+          const size_t base = ((size_t)e.unit_base * kMaxStat + i) * kTile + t;
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b)
+            x[k][b] = i < e.n_stat && u0 + b < nu
+                          ? __ldcg(p.part1 + base + (size_t)(u0 + b) * kStride)
+                          : make_float2(-INFINITY, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) acc[k] = lse_merge(acc[k], x[k][b]);
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int i = wg + 2 * k;
         const int tok = si.q0 + (e.stat0 + i) * p.tokq + t / p.G;
-        if (t >= p.tokq * p.G || tok >= si.len) continue;
-        float2 acc = make_float2(-INFINITY, 0.f);
-        for (int u0 = 0; u0 < e.n_units; u0 += kBatch) {
-          float2 x[kBatch];
+        if (i < e.n_stat && t < p.tokq * p.G && tok < si.len)
+          write_row_bias(p, si, g, tok, t % p.G, acc[k].x + log2f(acc[k].y));
+      }
+    } else {
+      float acc[2] = {0.f, 0.f};
+      for (int u0 = 0; u0 < nu; u0 += kBatch) {
+        float x[2][kBatch];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int i = wg + 2 * k;
+          const size_t base = ((size_t)e.unit_base * kMaxStat + i) * kTile + t;
 #pragma unroll
           for (int b = 0; b < kBatch; ++b)
-            x[b] = u0 + b < e.n_units ? __ldcg(p.part1 + base + (size_t)(u0 + b) * kStride)
-                                      : make_float2(-INFINITY, 0.f);
-#pragma unroll
-          for (int b = 0; b < kBatch; ++b) acc = lse_merge(acc, x[b]);
+            x[k][b] = i < e.n_stat && u0 + b < nu
+                          ? __ldcg(p.part2 + base + (size_t)(u0 + b) * kStride) : 0.f;
         }
-        write_row_bias(p, si, g, tok, t % p.G, acc.x + log2f(acc.y));
-      } else {
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) acc[k] += x[k][b];
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int i = wg + 2 * k;
         const int key = (e.stat0 + i) * kTile + t;
-        float sum = 0.f;
-        for (int u0 = 0; u0 < e.n_units; u0 += kBatch) {
-          float x[kBatch];
-#pragma unroll
-          for (int b = 0; b < kBatch; ++b)
-            x[b] = u0 + b < e.n_units ? __ldcg(p.part2 + base + (size_t)(u0 + b) * kStride) : 0.f;
-#pragma unroll
-          for (int b = 0; b < kBatch; ++b) sum += x[b];
-        }
-        if (key < si.len) p.scores[(size_t)g * p.T + si.start + key] = sum;
+        if (i < e.n_stat && key < si.len) p.scores[(size_t)g * p.T + si.start + key] = acc[k];
       }
     }
   }
@@ -635,16 +661,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_proxy_async_smem();
   if (warp == kMmaWarp) tmem_alloc(s.tmem_slot, kTmemCols);
   if (warp == kProducerWarp && lane == 0) { prefetch_tensormap(&tmQ); prefetch_tensormap(&tmK); }
-  pdl_allow_next();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s.tmem_slot;
-  pdl_wait();   // the plan (and Q, K) written by earlier kernels are visible from here
+  // Pass 1 waits for the planner (and whatever wrote Q, K) before anything,
+  // then lets pass 2 launch: from then on the plan, Q and K are complete, so
+  // pass 2's copy and MMA warps start on them at once; only its epilogue
+  // waits (below) for pass 1's row biases.
+  if (p1) {
+    pdl_wait();
+    pdl_allow_next();
+  }
 
   UnitIter it;
   const bool have = it.init(E, p1 ? H->n_e1 : H->n_e2, p1 ? H->s1 : H->s2,
-                            p1 ? H->p1 : H->p2, blockIdx.x);
+                            p1 ? H->p1 : H->p2, blockIdx.x,
+                            (p1 ? H->aligned1 : H->aligned2) != 0);
   if (warp >= kProducerWarp) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
     if (have && warp == kProducerWarp) {
@@ -656,6 +689,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpilogue));
+    if (!p1) {
+      pdl_wait();
+      pdl_allow_next();
+    }
     if (have) epilogue<D>(p, s, E, it, tmem);
   }
   tc_fence_before();

@@ -6,8 +6,13 @@
 
 namespace waits {
 
-// CTA `cta` of `P` owns global steps [ceil(cta*S/P), ceil((cta+1)*S/P)); a
-// maximal run of them inside one entry is a unit.
+// Two ways to split a pass's steps over its P CTAs, chosen by the planner:
+//  * by global step: CTA `cta` owns global steps [ceil(cta*S/P),
+//    ceil((cta+1)*S/P)); a maximal run of them inside one entry is a unit,
+//    so a CTA may hold pieces of several entries;
+//  * entry by entry ("aligned"): entry e owns CTAs [first_cta, first_cta +
+//    n_units), which split its steps evenly; every CTA has exactly one unit,
+//    so none pays for a second set of stationary tiles.
 struct UnitIter {
   const Entry* E;
   int nE;
@@ -16,9 +21,23 @@ struct UnitIter {
   int64_t pos;    // next global step
   int cta;
 
-  __device__ bool init(const Entry* E_, int nE_, int64_t S, int P, int cta_) {
+  __device__ bool init(const Entry* E_, int nE_, int64_t S, int P, int cta_, bool aligned) {
     E = E_; nE = nE_; cta = cta_;
     if (cta >= P || nE <= 0 || S <= 0) return false;
+    if (aligned) {
+      int a = 0, b = nE - 1;
+      while (a < b) {
+        const int m = (a + b + 1) / 2;
+        if (E[m].first_cta <= cta) a = m; else b = m - 1;
+      }
+      const Entry& en = E[a];
+      const int64_t u = cta - en.first_cta, nu = en.n_units, n = en.n_steps;
+      if (u < 0 || u >= nu) return false;
+      e = a;
+      pos = en.sbase + u * n / nu;
+      hi = en.sbase + (u + 1) * n / nu;
+      return pos < hi;
+    }
     const int64_t lo = ((int64_t)cta * S + P - 1) / P;
     hi = ((int64_t)(cta + 1) * S + P - 1) / P;
     if (lo >= hi) return false;

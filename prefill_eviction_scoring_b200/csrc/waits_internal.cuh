@@ -63,7 +63,8 @@ struct PlanHeader {
   int32_t p1, p2;      // CTAs that own work per pass (<= grid)
   int32_t pad0;
   int64_t s1, s2;      // total steps per pass
-  int32_t pad[4];
+  int32_t aligned1, aligned2;  // per pass: CTAs split entry by entry (1) or by global step (0)
+  int32_t pad[2];
 };
 
 // ------------------------------------------------------ workspace layout ---
@@ -136,8 +137,19 @@ __device__ inline int first_active_row(int N, float a, int b) {
 
 // --------------------------------------------------------- block scans ---
 // Exclusive prefix sum over the threads of a block (a multiple of 32, <= 1024).
+// A one-warp block scans with shuffles alone, without barriers.
 __device__ inline int64_t block_exclusive_scan(int64_t v, int64_t* total, int64_t* sh /*[32]*/) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (blockDim.x == 32) {
+    int64_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    *total = __shfl_sync(0xffffffffu, x, 31);
+    return x - v;
+  }
   int64_t x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
