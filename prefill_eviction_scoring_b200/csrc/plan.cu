@@ -15,7 +15,7 @@ __device__ inline int ceil_div(int x, int y) { return (x + y - 1) / y; }
 
 // Number of stationary groups per (sequence, KV head) for each pass.
 __device__ inline int groups_p1(const SeqInfo& si) {
-  return si.len > si.q0 ? ceil_div(si.nqt, kMaxStat) : 0;
+  return si.len > si.q0 ? ceil_div(si.nqt, kMaxStat1) : 0;
 }
 __device__ inline int groups_p2(const SeqInfo& si) {
   if (si.len <= si.q0) return 0;
@@ -34,8 +34,8 @@ __device__ void fill_entry_p1(int tokq, const SeqInfo& si, int s, int local, Ent
   e.g = local / ng;
   e.grp = local % ng;
   e.mode = kModeP1;
-  e.stat0 = e.grp * kMaxStat;
-  e.n_stat = min(kMaxStat, si.nqt - e.stat0);
+  e.stat0 = e.grp * kMaxStat1;
+  e.n_stat = min(kMaxStat1, si.nqt - e.stat0);
   const int last = qtile_last_token(si, e.stat0 + e.n_stat - 1, tokq);
   e.step0 = 0;
   e.n_steps = last / kTile + 1;

@@ -47,17 +47,21 @@ constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s after an abort
 constexpr int kBarWG0 = 1;                           // named barriers: 1, 2 per WG,
 constexpr int kBarAll = 3;                           // 3 for both WGs
 
-template <int D>
+// Shared-memory plan per head dim and pass: pass 1 holds 2 stationary Q
+// tiles and streams K through 4 stages (d = 128); pass 2 holds up to 4
+// stationary tiles with 2 stages.
+template <int D, int PASS>
 struct Cfg {
   static constexpr int kSub = D / 64;                    // 128-byte column blocks
   static constexpr int kSubBytes = kTile * 128;          // 16 KB
   static constexpr int kTileBytes = kSub * kSubBytes;
-  static constexpr int kStages = D == 128 ? 2 : 4;
+  static constexpr int kStat = PASS == 1 ? kMaxStat1 : kMaxStat;
+  static constexpr int kStages = (D == 128 ? 2 : 4) * (PASS == 1 ? 2 : 1);
   static constexpr int kKSteps = D / 16;
   static constexpr size_t kFloats = kMaxStat * kTile            // stationary Q biases
                                     + kWGs * 2 * kTile           // streamed Q biases
                                     + 2 * kWGs * kMaxStat * kTile;  // per-WG state
-  static constexpr size_t kSmem = 1024 + (size_t)(kMaxStat + kStages) * kTileBytes +
+  static constexpr size_t kSmem = 1024 + (size_t)(kStat + kStages) * kTileBytes +
                                   kFloats * sizeof(float) + 256;
 };
 
@@ -80,14 +84,14 @@ struct Smem {
   int* last;
 };
 
-template <int D>
+template <int D, int PASS>
 __device__ Smem carve(uint8_t* raw) {
-  using C = Cfg<D>;
+  using C = Cfg<D, PASS>;
   Smem s;
   const uint32_t a = smem_addr(raw);
   uint8_t* base = raw + ((1024u - (a & 1023u)) & 1023u);
   s.stat = base;
-  s.strm = s.stat + kMaxStat * C::kTileBytes;
+  s.strm = s.stat + C::kStat * C::kTileBytes;
   s.bias_stat = reinterpret_cast<float*>(s.strm + C::kStages * C::kTileBytes);
   s.bias_strm = s.bias_stat + kMaxStat * kTile;
   s.st_m = s.bias_strm + kWGs * 2 * kTile;
@@ -118,11 +122,11 @@ __device__ inline void pair_tiles(const Entry& e, int o, int i, int& j, int& kt)
 }
 
 // ------------------------------------------------------------ producer ---
-template <int D>
+template <int D, int PASS>
 __device__ void load_tile(const CUtensorMap* tmQ, const CUtensorMap* tmK, uint8_t* dst,
                           uint64_t* bar, const PassArgs& p, const SeqInfo& si, int g, bool is_q,
                           int idx) {
-  using C = Cfg<D>;
+  using C = Cfg<D, PASS>;
 #pragma unroll
   for (int sb = 0; sb < C::kSub; ++sb) {
     if (is_q)
@@ -133,10 +137,10 @@ __device__ void load_tile(const CUtensorMap* tmQ, const CUtensorMap* tmK, uint8_
   }
 }
 
-template <int D>
+template <int D, int PASS>
 __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const PassArgs& p,
                          const Smem& s, const Entry* E, UnitIter it) {
-  using C = Cfg<D>;
+  using C = Cfg<D, PASS>;
   const uint32_t q_bytes = (uint32_t)(D * 2 * p.G * p.tokq);
   const uint32_t k_bytes = (uint32_t)(D * 2 * kTile);
   int stage = 0;
@@ -154,7 +158,7 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const P
     if (!mbar_wait(s.stat_empty, uph ^ 1u, s.abort, p.status, kWaitLimitNs)) goto out;
     mbar_arrive_expect_tx(s.stat_full, (sq ? q_bytes : k_bytes) * (uint32_t)e.n_stat);
     for (int i = 0; i < e.n_stat; ++i)
-      load_tile<D>(tmQ, tmK, s.stat + i * C::kTileBytes, s.stat_full, p, si, e.g, sq,
+      load_tile<D, PASS>(tmQ, tmK, s.stat + i * C::kTileBytes, s.stat_full, p, si, e.g, sq,
                    e.stat0 + i);
     stat_issued = 1;
     stat_ph = uph;
@@ -162,7 +166,7 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const P
     for (int st = st0; st < st1; ++st) {
       if (!mbar_wait(&s.empty[stage], sph ^ 1u, s.abort, p.status, kWaitLimitNs)) goto out;
       mbar_arrive_expect_tx(&s.full[stage], sq ? k_bytes : q_bytes);
-      load_tile<D>(tmQ, tmK, s.strm + stage * C::kTileBytes, &s.full[stage], p, si, e.g, !sq,
+      load_tile<D, PASS>(tmQ, tmK, s.strm + stage * C::kTileBytes, &s.full[stage], p, si, e.g, !sq,
                    e.step0 + st);
       issued[stage] = 1;
       issued_ph[stage] = sph;
@@ -183,10 +187,10 @@ out:
 // Pairs of stationary slot i go to epilogue warpgroup i % 2, so both groups
 // work on the same streamed tile and the next one is prefetched meanwhile.
 // Each group owns two TMEM buffers.
-template <int D>
+template <int D, int PASS>
 __device__ void mma_issuer(const PassArgs& p, const Smem& s, const Entry* E, UnitIter it,
                            uint32_t tmem) {
-  using C = Cfg<D>;
+  using C = Cfg<D, PASS>;
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
   int stage = 0;
   uint32_t sph = 0, uph = 0;
@@ -456,7 +460,7 @@ __device__ inline float2 lse_merge(float2 x, float2 y) {
   return make_float2(M, x.y * ex2_approx(x.x - M) + y.y * ex2_approx(y.x - M));
 }
 
-template <int D>
+template <int D, int PASS>
 __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitIter it,
                          uint32_t tmem) {
   const int tid = threadIdx.x;               // 0..255
@@ -474,7 +478,7 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
     const int g = e.g;
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};   // P1 row state / P2K sums
     bar_sync(kBarAll, kEpiThreads);   // the previous unit's shared data is no longer read
-    if (e.mode == kModeP2Q) {
+    if (PASS == 2 && e.mode == kModeP2Q) {
       for (int i = wg; i < e.n_stat; i += kWGs)
         s.bias_stat[i * kTile + t] = qrow_bias(p, si, g, e.stat0 + i, t);
       bar_sync(kBarAll, kEpiThreads);
@@ -484,7 +488,7 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
       const int sb = sstep & 1;
       ++sstep;
       float* bias_o = s.bias_strm + sb * kTile;
-      if (e.mode == kModeP2K) {
+      if (PASS == 2 && e.mode == kModeP2K) {
         if (wg == 0) bias_o[t] = qrow_bias(p, si, g, o, t);
         bar_sync(kBarAll, kEpiThreads);
       }
@@ -508,7 +512,7 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.tempty[buf]);
-        if (e.mode == kModeP1) {
+        if (PASS == 1) {
           const int tok = si.q0 + j * p.tokq + t / p.G;
           const bool row_ok = t < p.tokq * p.G && tok < si.len;
           int nv = row_ok ? tok - kt * kTile + 1 : 0;
@@ -524,7 +528,7 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
           if (e.mode == kModeP2K) l[k] += a2; else col += a2;
         }
       }
-      if (e.mode == kModeP2Q) {
+      if (PASS == 2 && e.mode == kModeP2Q) {
         // the two warpgroups' halves of this key's column sum
         float* part = s.st_l + (sb * kWGs + wg) * kTile;
         part[t] = col;
@@ -540,8 +544,8 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
     // ---- unit results: each warpgroup writes the slots it owns
     const bool fail = bar_vote_or(kBarAll, kEpiThreads, !ok || *s.abort);
     if (fail) { ok = false; continue; }
-    if (e.mode == kModeP2Q) continue;
-    const bool p1 = e.mode == kModeP1;
+    if (PASS == 2 && e.mode == kModeP2Q) continue;
+    constexpr bool p1 = PASS == 1;
     if (e.n_units == 1) {
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
@@ -631,15 +635,15 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
   }
 }
 
-template <int D>
+template <int D, int PASS>
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
-                    const __grid_constant__ CUtensorMap tmK, PassArgs p, int pass) {
-  using C = Cfg<D>;
+                    const __grid_constant__ CUtensorMap tmK, PassArgs p) {
+  using C = Cfg<D, PASS>;
   extern __shared__ uint8_t smem_raw[];
-  const Smem s = carve<D>(smem_raw);
+  const Smem s = carve<D, PASS>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool p1 = pass == 1;
+  constexpr bool p1 = PASS == 1;
   const PlanHeader* H = p.hdr;
   const Entry* E = p1 ? p.e1 : p.e2;
 
@@ -655,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // padded rows of Q tiles are never written by TMA: keep them finite (zero)
   {
     uint4* z = reinterpret_cast<uint4*>(s.stat);
-    const int n = (kMaxStat + C::kStages) * C::kTileBytes / 16;
+    const int n = (C::kStat + C::kStages) * C::kTileBytes / 16;
     for (int i = threadIdx.x; i < n; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_smem();
@@ -681,10 +685,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= kProducerWarp) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
     if (have && warp == kProducerWarp) {
-      if (lane == 0) producer<D>(&tmQ, &tmK, p, s, E, it);
+      if (lane == 0) producer<D, PASS>(&tmQ, &tmK, p, s, E, it);
       __syncwarp();
     } else if (have && warp == kMmaWarp) {
-      if (lane == 0) mma_issuer<D>(p, s, E, it, tmem);
+      if (lane == 0) mma_issuer<D, PASS>(p, s, E, it, tmem);
       __syncwarp();
     }
   } else {
@@ -693,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       pdl_wait();
       pdl_allow_next();
     }
-    if (have) epilogue<D>(p, s, E, it, tmem);
+    if (have) epilogue<D, PASS>(p, s, E, it, tmem);
   }
   tc_fence_before();
   __syncthreads();
@@ -742,14 +746,19 @@ cudaError_t launch_d(const PassArgs& a, int grid, cudaStream_t st) {
   if (!make_map(&mq, a.Q, a.T, a.Hq, D, a.G, a.tokq) ||
       !make_map(&mk, a.K, a.T, a.Hkv, D, 1, kTile))
     return cudaErrorInvalidValue;
-  const size_t smem = Cfg<D>::kSmem;
-  cudaError_t err = cudaFuncSetAttribute(score_tc_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  if ((err = launch_pdl(score_tc_kernel<D>, dim3(grid), dim3(kThreads), smem, st, mq, mk, a, 1)) !=
-      cudaSuccess) {
+  const size_t smem1 = Cfg<D, 1>::kSmem, smem2 = Cfg<D, 2>::kSmem;
+  cudaError_t err;
+  if ((err = cudaFuncSetAttribute(score_tc_kernel<D, 1>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)) !=
+          cudaSuccess ||
+      (err = cudaFuncSetAttribute(score_tc_kernel<D, 2>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) !=
+          cudaSuccess)
+    return err;
+  if ((err = launch_pdl(score_tc_kernel<D, 1>, dim3(grid), dim3(kThreads), smem1, st, mq, mk,
+                        a)) != cudaSuccess) {
     cudaFuncAttributes fa{};
-    cudaFuncGetAttributes(&fa, score_tc_kernel<D>);
+    cudaFuncGetAttributes(&fa, score_tc_kernel<D, 1>);
     int dev = 0, optin = 0, regs = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -757,10 +766,10 @@ cudaError_t launch_d(const PassArgs& a, int grid, cudaStream_t st) {
     set_error_detail("scorer: regs %d, max threads %d, local %zu B, static smem %zu B, "
                      "dynamic %zu of opt-in %d B, block regs %d, threads %d",
                      fa.numRegs, fa.maxThreadsPerBlock, fa.localSizeBytes, fa.sharedSizeBytes,
-                     smem, optin, regs, kThreads);
+                     smem1, optin, regs, kThreads);
     return err;
   }
-  return launch_pdl(score_tc_kernel<D>, dim3(grid), dim3(kThreads), smem, st, mq, mk, a, 2);
+  return launch_pdl(score_tc_kernel<D, 2>, dim3(grid), dim3(kThreads), smem2, st, mq, mk, a);
 }
 
 }  // namespace

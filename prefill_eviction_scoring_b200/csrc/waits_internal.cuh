@@ -14,7 +14,8 @@ namespace waits {
 
 // ---------------------------------------------------------------- tiling ---
 constexpr int kTile = 128;      // keys per K tile; max packed rows per Q tile
-constexpr int kMaxStat = 4;     // stationary tiles held by one work unit
+constexpr int kMaxStat = 4;     // stationary tiles held by one work unit (at most)
+constexpr int kMaxStat1 = 2;    // pass 1: Q tiles per unit (leaves room for 4 K stages)
 constexpr int kMaxGrid = 1024;  // upper bound on persistent CTAs (sizing)
 constexpr int kPlanThreads = 256;
 
@@ -80,7 +81,7 @@ __host__ inline Layout make_layout(int64_t nseq, int64_t T, int64_t Hq, int64_t 
   Layout L{};
   const int64_t G = Hq / Hkv;
   const int64_t tokq = tokens_per_qtile((int)G);
-  L.max_e1 = Hkv * (T / (kMaxStat * tokq) + nseq);
+  L.max_e1 = Hkv * (T / (kMaxStat1 * tokq) + nseq);
   L.max_e2 = Hkv * (T / (kMaxStat * kTile) + nseq);
   L.max_u1 = L.max_e1 + kMaxGrid;
   L.max_u2 = L.max_e2 + kMaxGrid;
