@@ -40,6 +40,8 @@ UNIT = "tokens/s"
 CONFIG = "llama8b"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1590.0}
 KERNELS_PER_LAYER = 5   # plan, pass 1, pass 2, select, compact
+EVENT_EVERY = 8         # timed region: CUDA events around every 8th layer's scorer
+MUFU_EX2_PER_CLK_PER_SM = 16   # sm_100: 4 SFU lanes per SM sub-partition x 4
 # DRAM bytes (read + write) of one waits_score call on one llama8b layer, from
 # the ncu capture summarised in profiles/score_tc_select_llama8b_1layer.md
 # (both scorer passes).  Valid only for the scorer source it was taken on.
@@ -297,15 +299,16 @@ def run_ours(args):
 
     def step(evs=None, which="all"):
         """One pass of the path over every layer.  Events (if given) are
-        recorded around the scorer call, and with which="all" also around
-        select and compact; an event between two calls stops the next
-        kernel from starting early, so the timed region brackets only the
-        scorer."""
+        recorded around the scorer call of every EVENT_EVERY-th layer, and
+        with which="all" around every call; an event between two calls stops
+        the next kernel from starting early, so the timed region brackets
+        only a sample of the scorer calls."""
         for i, c in enumerate(calls):
-            if evs is not None:
+            timed = evs is not None and (which == "all" or i % EVENT_EVERY == 0)
+            if timed:
                 evs[i][0].record(stream)
             _lib.check("waits_score", c.score(lib, a, b, sp))
-            if evs is not None:
+            if timed:
                 evs[i][1].record(stream)
             _lib.check("waits_select", c.select(lib, R, sp))
             if evs is not None and which == "all":
@@ -341,7 +344,8 @@ def run_ours(args):
     D.barrier()
     ms = D.max(t0e.elapsed_time(t1e)) / K
     if args.kernel_events == "score":
-        t_score = D.max(statistics.mean(e[0].elapsed_time(e[1]) for s_ in evs for e in s_))
+        t_score = D.max(statistics.mean(e[0].elapsed_time(e[1]) for s_ in evs
+                                        for i, e in enumerate(s_) if i % EVENT_EVERY == 0))
 
     # select and compact durations: a few more steps with events around
     # every call (outside the timed region; they cut the overlap of calls)
@@ -365,16 +369,33 @@ def run_ours(args):
     pk, pk_kind = peaks()
     peak_t = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
     achieved_t = flops / (t_score / 1e3) / 1e12
+    timing = (f"CUDA events around the waits_score call of every {EVENT_EVERY}th layer in the "
+              "timed region" if args.kernel_events == "score" else
+              "CUDA events around waits_score in 5 steps after the timed region")
+    # The scorer's binding unit is the MUFU exponential: every active logit
+    # is exponentiated once per pass.  Peak = 16 ex2 per clock per SM (the
+    # SFU count of an sm_100 SM) x SMs x the maximum SM clock.
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    sm_max_ghz = float(pk.get("sm_max_mhz", 1965.0)) / 1e3
+    peak_exp = MUFU_EX2_PER_CLK_PER_SM * sm_count * sm_max_ghz        # G exp/s
+    exps = 2 * logits
+    achieved_exp = exps / (t_score / 1e3) / 1e9
     roof = {"kernel": "scorer (waits_score: planner + pass 1 + pass 2)",
-            "bound": "tensor", "achieved": round(achieved_t, 2), "peak": peak_t,
-            "unit": "TFLOP/s", "frac": round(achieved_t / peak_t, 4), "traffic": profiled_traffic(),
-            "peak_kind": f"bf16_tflops_sustained ({pk_kind})",
-            "flops_per_launch": flops, "launch_ms": round(t_score, 4),
-            "timing": "CUDA events around every waits_score call in the timed region"
-                      if args.kernel_events == "score" else
-                      "CUDA events around waits_score in 5 steps after the timed region"}
+            "bound": "alu", "achieved": round(achieved_exp, 1), "peak": round(peak_exp, 1),
+            "unit": "Gexp/s", "frac": round(achieved_exp / peak_exp, 4),
+            "traffic": profiled_traffic(),
+            "peak_kind": f"MUFU ex2: {MUFU_EX2_PER_CLK_PER_SM}/clk/SM x {sm_count} SMs x "
+                         f"{sm_max_ghz:.3f} GHz (unit count x measured max clock)",
+            "exps_per_launch": exps, "launch_ms": round(t_score, 4), "timing": timing}
+    hbm = float(pk.get("hbm_gbs"))
+    tensor_roof = {"kernel": "scorer, tensor view", "bound": "tensor",
+                   "achieved": round(achieved_t, 2), "peak": peak_t, "unit": "TFLOP/s",
+                   "frac": round(achieved_t / peak_t, 4),
+                   "peak_kind": f"bf16_tflops_sustained ({pk_kind})",
+                   "flops_per_launch": flops, "launch_ms": round(t_score, 4)}
     hbm = float(pk.get("hbm_gbs"))
     other = [
+        tensor_roof,
         {"kernel": "select", "bound": "hbm", "achieved": round(sel_b / (t_sel / 1e3) / 1e9, 1),
          "peak": hbm, "unit": "GB/s", "frac": round(sel_b / (t_sel / 1e3) / 1e9 / hbm, 4),
          "bytes_per_launch": sel_b, "launch_ms": round(t_sel, 4)},
