@@ -122,30 +122,45 @@ def peaks():
 
 # ------------------------------------------------------------- plumbing ---
 class Dist:
-    def __init__(self):
+    """One process per GPU (torchrun environment).  ``backend="gloo"`` runs
+    the same logic on CPU tensors (used by the multi-rank CPU tests)."""
+
+    def __init__(self, backend: str = "nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
         self.pg = None
 
+    @property
+    def cuda(self) -> bool:
+        return self.backend == "nccl"
+
+    def device(self):
+        return torch.device("cuda", self.local) if self.cuda else torch.device("cpu")
+
     def init(self):
-        torch.cuda.set_device(self.local)
+        if self.cuda:
+            torch.cuda.set_device(self.local)
         if self.world > 1:
             import torch.distributed as dist
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {"device_id": self.device()} if self.cuda else {}
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=180), **kw)
             self.pg = dist
 
     def barrier(self):
-        torch.cuda.synchronize()
+        if self.cuda:
+            torch.cuda.synchronize()
         if self.pg:
             self.pg.barrier()
-        torch.cuda.synchronize()
+        if self.cuda:
+            torch.cuda.synchronize()
 
     def max(self, x: float) -> float:
+        """Largest value over the ranks (every rank must call it)."""
         if not self.pg:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=self.device())
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
