@@ -2,34 +2,36 @@
 // the recent window [N-R, N) and the B-R highest scores of [0, N-R), ties to
 // the lower index, reported in ascending order.
 //
-// One 1024-thread CTA per (sequence, KV head).  Scores are mapped to a
-// monotone 32-bit image; the (B-R)-th largest image tau is found exactly by
-// a three-digit radix select (12 + 10 + 10 bits):
-//   1. one pass stages the pool's images in shared memory (16-byte loads)
-//      and histograms their top 12 bits;
-//   2. a block scan over the bins finds the bin that holds the (B-R)-th
-//      largest image;
-//   3. the images in that bin are copied to a candidate list, and the two
-//      lower digits are resolved on the candidates alone (on the whole pool
-//      when the bin holds more than the list's capacity);
-//   4. the output pass gives each thread 32 consecutive positions; one block
-//      scan of packed (above tau, equal to tau) counts per chunk of 32768
-//      positions places every kept position, threshold ties taken lowest
-//      index first.
-// Pools larger than the staging buffer are re-read from global memory
-// (L2) in each pass instead.
+// One thread-block cluster of kC CTAs per (sequence, KV head); CTA r of the
+// cluster owns slice r of the pool (a contiguous range of 16-byte groups).
+// Scores are mapped to a monotone 32-bit image; the (B-R)-th largest image
+// tau is found exactly by a radix select over digits of 12 + 10 + 10 bits.
+// For each digit every CTA histograms the images of its slice that carry the
+// digits found so far and sends the histogram to every CTA of the cluster
+// (distributed shared memory): the first digit's non-empty bins are added
+// into each CTA's cluster histogram; the second digit's into the CTA that
+// owns the bin (rank = bin / 128), from which every CTA gathers the sums
+// after the barrier; the third digit's histogram is stored per sending CTA.
+// Every CTA then finds the same digit itself, so a digit costs one cluster
+// barrier.  With the second and third digits each
+// CTA also sends how many of its images lie above the previous digit's bin;
+// from those counts and the per-CTA third-digit histograms every CTA knows
+// how many images above tau and equal to tau the slices before its own hold,
+// and places its kept positions with block scans, ties to tau taken lowest
+// index first.  The first pass stages the slice's images in shared memory,
+// so the later passes read no global memory.
 #include "waits_internal.cuh"
 
 namespace waits {
 namespace {
 
-constexpr int kSelThreads = 1024;
-constexpr int kGroupsPerThread = 8;              // output pass: 32 consecutive positions
-constexpr int kStageKeys = kSelThreads * kGroupsPerThread * 4;   // 32768 (128 KB)
+constexpr int kC = 8;                            // CTAs per cluster (portable maximum)
+constexpr int kSelThreads = 512;
+constexpr int kStageGroups = 2048;               // per CTA: 8192 staged images (32 KB)
 constexpr int kBins1 = 4096;                     // bits 20..31
-constexpr int kCopies = 4;                       // first-digit histograms (by warp % 4)
+constexpr int kCopies = 4;                       // local first-digit histograms (warp % 4)
 constexpr int kBins2 = 1024;                     // bits 10..19, then 0..9
-constexpr int kCand = 4096;                      // candidate list capacity
+constexpr int kMaxPer = kBins1 / kSelThreads;    // bins per thread in find_bin
 
 // Monotone map of fp32 to uint32: a < b (as floats, -0 == +0) iff
 // key(a) < key(b).  Scores from waits_score are >= 0, but waits_select takes
@@ -41,14 +43,49 @@ __device__ inline uint32_t order_key(float s) {
 }
 
 struct SelSmem {
-  uint32_t hist[kCopies * kBins1];
-  uint32_t cand[kCand];
+  uint32_t hist[kCopies * kBins1];   // this CTA's histograms
+  uint32_t g1[kBins1];               // the cluster's first-digit histogram
+  uint32_t g2[kBins2];               // the cluster's second-digit histogram (owned bins)
+  uint32_t h3[kC][kBins2];           // third-digit histogram of each slice
+  uint32_t above1[kC];               // per slice: images above the first digit's bin
+  uint32_t above2[kC];               // per slice: images in it, above the second's
   int64_t scan[32];
-  uint32_t digit;
+  uint32_t digit;                    // find_bin's result
   int32_t above;
-  int32_t count;
-  int32_t ncand;
 };
+
+// ---------------------------------------------------------- cluster ops ---
+__device__ inline uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA in the cluster; orders shared-memory writes
+// (local and remote) before the barrier with reads after it.
+__device__ inline void cluster_sync() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ inline uint32_t peer(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(r)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))), "r"(rank));
+  return r;
+}
+__device__ inline void peer_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ inline uint32_t peer_ld32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ inline void peer_st32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 // The pool seen as aligned 16-byte groups: group i holds positions
 // 4i - off .. 4i - off + 3 (off = misalignment of the first score in
@@ -56,7 +93,6 @@ struct SelSmem {
 struct Pool {
   const float* base;   // 16-byte aligned, = scores of position -off
   int off, pool, ngroups;
-  const uint4* stage;  // staged images, or null
   __device__ uint4 image(int i, float4 f) const {
     const int p = 4 * i - off;
     return make_uint4(p + 0 >= 0 && p + 0 < pool ? order_key(f.x) : 0u,
@@ -64,14 +100,9 @@ struct Pool {
                       p + 2 >= 0 && p + 2 < pool ? order_key(f.z) : 0u,
                       p + 3 >= 0 && p + 3 < pool ? order_key(f.w) : 0u);
   }
-  __device__ uint4 group(int i) const {
-    if (stage) return stage[swz(i)];
+  __device__ uint4 load(int i) const {
     return image(i, __ldg(reinterpret_cast<const float4*>(base) + i));
   }
-  // Staged slot of group i: the eight groups of each 128-byte block are
-  // permuted by bits 3..5 of i, so both 32 consecutive groups (passes 1-3)
-  // and groups 8t + j of threads t = 0..31 (output pass) hit all 32 banks.
-  __device__ static int swz(int i) { return i ^ ((i >> 3) & 7); }
   // validity of the four positions of group i, as bits
   __device__ uint32_t valid(int i) const {
     const int p = 4 * i - off;
@@ -87,26 +118,25 @@ __device__ inline uint32_t comp(const uint4& v, int e) {
 }
 
 // Find the bin (bins in descending order) holding the need-th largest image
-// among `nb` bins of sm.hist (summed over `copies` histograms of nb bins);
-// result in sm.digit / sm.above, the bin's count in sm.count.  nb / 1024
-// bins per thread (1 or 4).  Ends with a barrier.
-__device__ void find_bin(SelSmem& sm, int nb, int copies, int need) {
+// among the nb bins of h; result in sm.digit / sm.above.  Ends with a barrier.
+__device__ void find_bin(SelSmem& sm, const uint32_t* h, int nb, int need) {
   const int per = nb / kSelThreads;
   const int top = nb - 1 - (int)threadIdx.x * per;
-  uint32_t c[4] = {0, 0, 0, 0}, sum = 0;
-  for (int i = 0; i < per; ++i) {
-    for (int k = 0; k < copies; ++k) c[i] += sm.hist[k * nb + top - i];
+  uint32_t c[kMaxPer], sum = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxPer; ++i) {
+    c[i] = i < per ? h[top - i] : 0u;
     sum += c[i];
   }
   int64_t tot;
   const int64_t ex = block_exclusive_scan((int64_t)sum, &tot, sm.scan);
   if (ex < need && ex + sum >= need) {
     int64_t cum = ex;
-    for (int i = 0; i < per; ++i) {
-      if (cum + c[i] >= need) {
+#pragma unroll
+    for (int i = 0; i < kMaxPer; ++i) {
+      if (i < per && cum + c[i] >= need) {
         sm.digit = (uint32_t)(top - i);
         sm.above = (int)cum;
-        sm.count = (int)c[i];
         break;
       }
       cum += c[i];
@@ -119,63 +149,82 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const float* __restrict__ scores, const int32_t* __restrict__ cu, int nseq, int T,
     int Hkv, int R, int B, int32_t* __restrict__ idx, int32_t* __restrict__ kept_len,
     uint32_t* status) {
-  extern __shared__ uint4 stage_raw[];      // [kStageKeys / 4] staged groups, then SelSmem
-  SelSmem& sm = *reinterpret_cast<SelSmem*>(stage_raw + kStageKeys / 4);
+  extern __shared__ uint4 dyn_smem[];
+  uint4* stage = dyn_smem;                                     // [kStageGroups]
+  SelSmem& sm = *reinterpret_cast<SelSmem*>(dyn_smem + kStageGroups);
   const int tid = threadIdx.x;
+  const uint32_t rank = cluster_rank();
   pdl_allow_next();
+  // nothing here depends on the previous kernel: zero the histograms and
+  // meet the cluster (every CTA runs before any shared memory is shared)
+  for (int i = tid; i < kCopies * kBins1; i += kSelThreads) sm.hist[i] = 0u;
+  for (int i = tid; i < kBins1; i += kSelThreads) sm.g1[i] = 0u;
+  for (int i = tid; i < kBins2; i += kSelThreads) sm.g2[i] = 0u;
+  for (int i = tid; i < kC * kBins2; i += kSelThreads) (&sm.h3[0][0])[i] = 0u;
+  __syncthreads();
+  cluster_sync();
   pdl_wait();
-  const int s = blockIdx.x / Hkv, g = blockIdx.x % Hkv;
+  // every branch below is taken by all CTAs of a cluster alike
+  const int sg = blockIdx.x / kC;
+  const int s = sg / Hkv, g = sg % Hkv;
   const int lo = cu[s], hi = cu[s + 1];
   int32_t* out = idx + ((size_t)s * Hkv + g) * B;
   const bool bad = (s == 0 && lo != 0) || hi < lo || hi > T || (s == nseq - 1 && hi != T);
   if (bad) {
-    for (int j = tid; j < B; j += kSelThreads) out[j] = -1;
-    if (tid == 0) {
-      if (g == 0) kept_len[s] = 0;
-      if (status) atomicOr(status, WAITS_DEV_BAD_SEQLENS);
+    if (rank == 0) {
+      for (int j = tid; j < B; j += kSelThreads) out[j] = -1;
+      if (tid == 0) {
+        if (g == 0) kept_len[s] = 0;
+        if (status) atomicOr(status, WAITS_DEV_BAD_SEQLENS);
+      }
     }
     return;
   }
   const int N = hi - lo;
-  if (g == 0 && tid == 0) kept_len[s] = N < B ? N : B;
+  if (rank == 0 && g == 0 && tid == 0) kept_len[s] = N < B ? N : B;
   if (N <= B) {
-    for (int j = tid; j < B; j += kSelThreads) out[j] = j < N ? j : -1;
+    if (rank == 0)
+      for (int j = tid; j < B; j += kSelThreads) out[j] = j < N ? j : -1;
     return;
   }
   const int want = B - R;            // positions taken from the pool by score
   const int pool = N - R;            // > want because N > B
-  for (int j = tid; j < R; j += kSelThreads) out[want + j] = pool + j;   // recent window
+  if (rank == 0)
+    for (int j = tid; j < R; j += kSelThreads) out[want + j] = pool + j;   // recent window
   if (want == 0) return;
 
-  // ---- 1. stage the images (if they fit) and histogram the top 12 bits
   const float* sc = scores + (size_t)g * T + lo;
   Pool P;
   P.off = (int)((reinterpret_cast<uintptr_t>(sc) >> 2) & 3u);
   P.base = sc - P.off;
   P.pool = pool;
   P.ngroups = (pool + P.off + 3) / 4;
-  P.stage = nullptr;
-  const bool staged = 4 * P.ngroups <= kStageKeys;
-  for (int i = tid; i < kCopies * kBins1; i += kSelThreads) sm.hist[i] = 0u;
-  if (tid == 0) sm.ncand = 0;
-  __syncthreads();
+  // this CTA's slice of groups
+  const int g_lo = (int)((int64_t)P.ngroups * rank / kC);
+  const int g_hi = (int)((int64_t)P.ngroups * (rank + 1) / kC);
+  const bool staged = g_hi - g_lo <= kStageGroups;
+  auto group = [&](int i) { return staged ? stage[i - g_lo] : P.load(i); };
+  uint32_t* loc2 = sm.hist + kBins1;       // this slice's second-digit histogram
+  uint32_t* loc3 = sm.hist + 2 * kBins1;   // this slice's third-digit histogram
+
+  // ---- first digit: stage the slice and histogram its top 12 bits
   {
     uint32_t* hist = sm.hist + ((tid >> 5) & (kCopies - 1)) * kBins1;
     constexpr int kUnroll = 4;
-    for (int i0 = 0; i0 < P.ngroups; i0 += kUnroll * kSelThreads) {
+    for (int i0 = g_lo; i0 < g_hi; i0 += kUnroll * kSelThreads) {
       float4 f[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int i = i0 + u * kSelThreads + tid;
-        f[u] = i < P.ngroups ? __ldg(reinterpret_cast<const float4*>(P.base) + i)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        f[u] = i < g_hi ? __ldg(reinterpret_cast<const float4*>(P.base) + i)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int i = i0 + u * kSelThreads + tid;
-        if (i < P.ngroups) {
+        if (i < g_hi) {
           const uint4 v = P.image(i, f[u]);
-          if (staged) stage_raw[Pool::swz(i)] = v;
+          if (staged) stage[i - g_lo] = v;
           const uint32_t ok = P.valid(i);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
@@ -184,91 +233,128 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
       }
     }
   }
-  if (staged) P.stage = stage_raw;
   __syncthreads();
+  // copy 0 keeps this slice's histogram (summed over the copies); its
+  // non-empty bins are added into every CTA's cluster histogram
+  for (int b = tid; b < kBins1; b += kSelThreads) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int k = 0; k < kCopies; ++k) c += sm.hist[k * kBins1 + b];
+    sm.hist[b] = c;
+    if (c) {
+#pragma unroll
+      for (int r = 0; r < kC; ++r) peer_add(peer(&sm.g1[b], (uint32_t)r), c);
+    }
+  }
+  cluster_sync();   // every CTA holds the cluster's first-digit histogram
+  find_bin(sm, sm.g1, kBins1, want);
+  const uint32_t d1 = sm.digit;
+  int need = want - sm.above;
 
-  // ---- 2. threshold bin of the first digit
-  int need = want;
-  find_bin(sm, kBins1, kCopies, need);
-  uint32_t prefix = sm.digit << 20, pmask = 0xFFF00000u;
+  // ---- second digit: bits 10..19 of the images in bin d1
+  {
+    uint32_t above = 0;
+    for (int b = tid; b < kBins1; b += kSelThreads) above += (uint32_t)b > d1 ? sm.hist[b] : 0u;
+    for (int b = tid; b < kBins2; b += kSelThreads) loc2[b] = 0u;
+    int64_t tot;
+    block_exclusive_scan((int64_t)above, &tot, sm.scan);   // barrier: loc2 is zero
+    if (tid < kC) peer_st32(peer(&sm.above1[rank], (uint32_t)tid), (uint32_t)tot);
+    for (int i = g_lo + tid; i < g_hi; i += kSelThreads) {
+      const uint4 v = group(i);
+      const uint32_t ok = P.valid(i);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t x = comp(v, e);
+        if (((ok >> e) & 1u) && (x >> 20) == d1) atomicAdd(&loc2[(x >> 10) & (kBins2 - 1)], 1u);
+      }
+    }
+    __syncthreads();
+    for (int b = tid; b < kBins2; b += kSelThreads) {
+      const uint32_t c = loc2[b];
+      if (c) peer_add(peer(&sm.g2[b], (uint32_t)(b / (kBins2 / kC))), c);
+    }
+  }
+  cluster_sync();   // the owners hold the second-digit histogram; every CTA the counts
+  // gather the owners' bins (into loc3, zeroed again below)
+  for (int b = tid; b < kBins2; b += kSelThreads)
+    loc3[b] = peer_ld32(peer(&sm.g2[b], (uint32_t)(b / (kBins2 / kC))));
+  __syncthreads();
+  find_bin(sm, loc3, kBins2, need);
+  const uint32_t d2 = sm.digit;
   need -= sm.above;
-  const int nbin = sm.count;
+  const uint32_t pre2 = (d1 << 10) | d2;   // top 22 bits of tau
+
+  // ---- third digit: bits 0..9 of the images carrying pre2, per slice
+  {
+    uint32_t above = 0;
+    for (int b = tid; b < kBins2; b += kSelThreads) above += (uint32_t)b > d2 ? loc2[b] : 0u;
+    for (int b = tid; b < kBins2; b += kSelThreads) loc3[b] = 0u;
+    int64_t tot;
+    block_exclusive_scan((int64_t)above, &tot, sm.scan);   // barrier: loc3 is zero
+    if (tid < kC) peer_st32(peer(&sm.above2[rank], (uint32_t)tid), (uint32_t)tot);
+    for (int i = g_lo + tid; i < g_hi; i += kSelThreads) {
+      const uint4 v = group(i);
+      const uint32_t ok = P.valid(i);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t x = comp(v, e);
+        if (((ok >> e) & 1u) && (x >> 10) == pre2) atomicAdd(&loc3[x & (kBins2 - 1)], 1u);
+      }
+    }
+    __syncthreads();
+    for (int b = tid; b < kBins2; b += kSelThreads) {
+      const uint32_t c = loc3[b];
+      if (c) {
+#pragma unroll
+        for (int r = 0; r < kC; ++r) peer_st32(peer(&sm.h3[rank][b], (uint32_t)r), c);
+      }
+    }
+  }
+  cluster_sync();   // every CTA holds every slice's third-digit histogram; no remote
+                    // shared-memory access follows
+  // cluster histogram of the third digit (into loc2, no longer needed)
+  for (int b = tid; b < kBins2; b += kSelThreads) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int r = 0; r < kC; ++r) c += sm.h3[r][b];
+    loc2[b] = c;
+  }
   __syncthreads();
-
-  // ---- 3. the two lower digits, on the bin's candidates when they fit
-  const bool listed = nbin <= kCand;
-  if (listed) {
-    for (int i0 = 0; i0 < P.ngroups; i0 += kSelThreads) {    // whole warps iterate
-      const int i = i0 + tid;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      uint32_t ok = 0;
-      if (i < P.ngroups) { v = P.group(i); ok = P.valid(i); }
-      uint32_t take = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        take |= (uint32_t)(((ok >> e) & 1u) && (comp(v, e) & pmask) == prefix) << e;
-      // one shared-memory atomic per warp for the whole warp's candidates
-      const int n = __popc(take);
-      int incl = n;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if ((tid & 31) >= o) incl += y;
-      }
-      const int wtot = __shfl_sync(0xffffffffu, incl, 31);
-      int base = 0;
-      if ((tid & 31) == 31 && wtot) base = atomicAdd(&sm.ncand, wtot);
-      base = __shfl_sync(0xffffffffu, base, 31) + incl - n;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if ((take >> e) & 1u) {
-          if (base < kCand) sm.cand[base] = comp(v, e);    // base < nbin <= kCand
-          ++base;
-        }
-    }
-    __syncthreads();
+  find_bin(sm, loc2, kBins2, need);
+  const uint32_t d3 = sm.digit;
+  need -= sm.above;
+  const uint32_t tau = (pre2 << 10) | d3;   // need = ties of tau to keep, lowest index first
+  // images above tau (high half) and equal to tau (low half) in the slices
+  // before this one
+  int64_t before = 0;
+  for (uint32_t r = 0; r < rank; ++r) {
+    if (tid == 0)
+      before += ((int64_t)sm.above1[r] + sm.above2[r]) * (int64_t(1) << 32) + sm.h3[r][d3];
+    for (int b = tid; b < kBins2; b += kSelThreads)
+      before += (uint32_t)b > d3 ? (int64_t)sm.h3[r][b] << 32 : 0;
   }
-#pragma unroll 1
-  for (int shift = 10; shift >= 0; shift -= 10) {
-    for (int i = tid; i < kBins2; i += kSelThreads) sm.hist[i] = 0u;
-    __syncthreads();
-    if (listed) {
-      for (int q = tid; q < nbin; q += kSelThreads) {
-        const uint32_t x = sm.cand[q];
-        if ((x & pmask) == prefix) atomicAdd(&sm.hist[(x >> shift) & 1023u], 1u);
-      }
-    } else {
-      for (int i = tid; i < P.ngroups; i += kSelThreads) {
-        const uint4 v = P.group(i);
+  int64_t gt_base, eq_base;
+  {
+    int64_t tot;
+    block_exclusive_scan(before, &tot, sm.scan);
+    gt_base = tot >> 32;
+    eq_base = tot & 0xFFFFFFFFll;
+  }
+
+
+  // ---- ascending positions: rounds of kOutGroups * kSelThreads consecutive
+  // groups (kOutGroups per thread), one block scan of packed (above tau,
+  // equal to tau) counts per round
+  constexpr int kOutGroups = 2;
+  for (int i0 = g_lo; i0 < g_hi; i0 += kOutGroups * kSelThreads) {
+    const int ib = i0 + kOutGroups * tid;
+    uint32_t gtm = 0, eqm = 0;     // bit 4j + e: position 4(ib + j) + e - off
+#pragma unroll
+    for (int j = 0; j < kOutGroups; ++j) {
+      const int i = ib + j;
+      if (i < g_hi) {
+        const uint4 v = group(i);
         const uint32_t ok = P.valid(i);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t x = comp(v, e);
-          if (((ok >> e) & 1u) && (x & pmask) == prefix)
-            atomicAdd(&sm.hist[(x >> shift) & 1023u], 1u);
-        }
-      }
-    }
-    __syncthreads();
-    find_bin(sm, kBins2, 1, need);
-    prefix |= sm.digit << shift;
-    pmask |= 1023u << shift;
-    need -= sm.above;
-    __syncthreads();
-  }
-  const uint32_t tau = prefix;   // need = ties of tau to keep, lowest index first
-
-  // ---- 4. ascending output: thread t walks groups 8t .. 8t+7 of a chunk of
-  // 8192 groups (32 consecutive positions); one block scan per chunk
-  int64_t gt_base = 0, eq_base = 0;
-  for (int c0 = 0; c0 < P.ngroups; c0 += kSelThreads * kGroupsPerThread) {
-    const int g0 = c0 + kGroupsPerThread * tid;
-    uint32_t gtm = 0, eqm = 0;     // bit 4j + e: position 4(g0 + j) + e - off
-#pragma unroll
-    for (int j = 0; j < kGroupsPerThread; ++j) {
-      if (g0 + j < P.ngroups) {
-        const uint4 v = P.group(g0 + j);
-        const uint32_t ok = P.valid(g0 + j);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t x = comp(v, e);
@@ -277,12 +363,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
         }
       }
     }
-    // packed counts: above tau in the high half, ties in the low half
     const int64_t mine = ((int64_t)__popc(gtm) << 32) | (int64_t)__popc(eqm);
     int64_t tot;
     const int64_t ex = block_exclusive_scan(mine, &tot, sm.scan);
-    int64_t gt_before = gt_base + (ex >> 32), eq_before = eq_base + (ex & 0xFFFFFFFFll);
-    const int p0 = 4 * g0 - P.off;
+    const int64_t gt_before = gt_base + (ex >> 32), eq_before = eq_base + (ex & 0xFFFFFFFFll);
+    const int p0 = 4 * ib - P.off;
     uint32_t any = gtm | eqm;
     while (any) {
       const int b = __ffs(any) - 1;
@@ -305,14 +390,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int T, int Hkv,
                           int R, int B, int32_t* idx, int32_t* kept_len, uint32_t* status,
                           cudaStream_t s) {
-  const int64_t grid = (int64_t)nseq * Hkv;
+  const int64_t grid = (int64_t)nseq * Hkv * kC;
   if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  const int dyn = kStageKeys * (int)sizeof(uint32_t) + (int)sizeof(SelSmem);
+  const int dyn = kStageGroups * (int)sizeof(uint4) + (int)sizeof(SelSmem);
   cudaError_t err = cudaFuncSetAttribute(select_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
   if (err != cudaSuccess) return err;
-  return launch_pdl(select_kernel, dim3((unsigned)grid), dim3(kSelThreads), (size_t)dyn, s,
-                    scores, cu, nseq, T, Hkv, R, B, idx, kept_len, status);
+  return launch_pdl_cluster(select_kernel, dim3((unsigned)grid), dim3(kSelThreads), kC,
+                            (size_t)dyn, s, scores, cu, nseq, T, Hkv, R, B, idx, kept_len,
+                            status);
 }
 
 }  // namespace waits
