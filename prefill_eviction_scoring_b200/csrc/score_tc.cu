@@ -245,28 +245,24 @@ out:
 }
 
 // ------------------------------------------------------------ epilogue ---
-// 128 accumulator columns of this thread's TMEM lane.  The wait names every
-// register so no use of them can be scheduled before the data has arrived.
+// 128 accumulator columns of this thread's TMEM lane: the load and its wait
+// in one statement, so no use of the registers can be scheduled before the
+// data has arrived and the registers need no read-write operands (which can
+// cost a copy of each).
 struct Cols {
   uint32_t r[128];
-  __device__ void load(uint32_t taddr) {
-    uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
-    uint32_t(&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
-    uint32_t(&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
-    uint32_t(&d)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
-    tmem_ld32(taddr, a);
-    tmem_ld32(taddr + 32, b);
-    tmem_ld32(taddr + 64, c);
-    tmem_ld32(taddr + 96, d);
-  }
-  __device__ void wait() {
-#define W8(b) "+r"(r[b]), "+r"(r[b + 1]), "+r"(r[b + 2]), "+r"(r[b + 3]), "+r"(r[b + 4]), \
-              "+r"(r[b + 5]), "+r"(r[b + 6]), "+r"(r[b + 7])
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : W8(0), W8(8), W8(16), W8(24), W8(32), W8(40), W8(48), W8(56), W8(64), W8(72),
-                   W8(80), W8(88), W8(96), W8(104), W8(112), W8(120)
-                 :
-                 : "memory");
+  __device__ void load_wait(uint32_t taddr) {
+#define W8(b) "=r"(r[b]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), \
+              "=r"(r[b + 5]), "=r"(r[b + 6]), "=r"(r[b + 7])
+    asm volatile(
+        "{\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "}"
+        : W8(0), W8(8), W8(16), W8(24), W8(32), W8(40), W8(48), W8(56),
+          W8(64), W8(72), W8(80), W8(88), W8(96), W8(104), W8(112), W8(120)
+        : "r"(taddr)
+        : "memory");
 #undef W8
   }
 };
@@ -279,9 +275,10 @@ __device__ inline float hsum8(const float2 (&a)[4]) {
 
 // Column pairs whose exponential runs on the FMA pipe instead of the MUFU
 // (which does 16 ex2 per clock per SM and bounds the unmasked passes): bit
-// (pair index mod 8) of this mask.  Two in eight, spread out, measured best;
-// more makes the warps issue-bound.
-constexpr uint32_t kPolyPairs = 0x88u;
+// (pair index mod 8) of this mask.  One in eight measured best here (the
+// epilogue is latency-bound rather than MUFU-bound in this kernel; two in
+// eight was within 1.5%, three in eight 6% slower).
+constexpr uint32_t kPolyPairs = 0x80u;
 __device__ constexpr bool poly_col(int c) { return (kPolyPairs >> ((c >> 1) & 7)) & 1u; }
 
 // 2^x for a pair of fp32 values on the FMA/ALU pipes (Cody-Waite split plus
@@ -507,8 +504,7 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
         if (!ok) continue;
         tc_fence_after();
         Cols v;
-        v.load(lane_addr + (uint32_t)(buf * kTile));
-        v.wait();
+        v.load_wait(lane_addr + (uint32_t)(buf * kTile));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.tempty[buf]);
