@@ -152,7 +152,7 @@ __device__ void plan_pass(const Seqs& S, int nseq, int tokq, int n, int grid, En
     ub += tot;
     if (i < n) {
       out[i] = e;
-      counters[i] = 0u;
+      if (counters) counters[i] = 0u;
     }
   }
   *steps = Stot;
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs p) {
   int64_t S1 = 0, S2 = 0;
   int U1 = 0, U2 = 0, P1 = 0, P2 = 0, A1 = 0, A2 = 0;
   if (!overflow) {
-    plan_pass<true>(S, p.nseq, p.tokq, (int)c1, p.grid, p.e1, p.c1, p.max_u1, sh, &S1, &U1,
+    plan_pass<true>(S, p.nseq, p.tokq, (int)c1, p.grid, p.e1, nullptr, p.max_u1, sh, &S1, &U1,
                     &P1, &A1, &overflow);
     plan_pass<false>(S, p.nseq, p.tokq, (int)c2, p.grid, p.e2, p.c2, p.max_u2, sh, &S2, &U2,
                      &P2, &A2, &overflow);

@@ -4,9 +4,10 @@
 // key k is the accumulative attention it receives, each query row q weighted
 // by the forgetting curve w[q].  Read as causal softmax(QK^T / sqrt(d)) summed
 // over the query heads of a KV group:
-//   pass 1  bias[q,h] = log2 w[q] - log2 sum_{k<=q} 2^(x[q,k]),
-//           x = (Q.K) * log2(e) / sqrt(d)
-//   pass 2  s[g,k]    = sum_{h in g} sum_{q>=k} 2^(x[q,k] + bias[q,h])
+//   pass 1  per row (q, h): sum_{k<=q} 2^(x[q,k]), x = (Q.K) * log2(e) / sqrt(d),
+//           as (reference max, sum) partials of the CTAs sharing the row
+//   pass 2  bias[q,h] = log2 w[q] - log2 of the merged sum, then
+//           s[g,k]    = sum_{h in g} sum_{q>=k} 2^(x[q,k] + bias[q,h])
 // Rows whose fp32 weight is exactly 0 are never visited (the planner starts
 // each sequence at its first non-zero row).
 //
@@ -435,26 +436,38 @@ __device__ inline bool bar_vote_or(int id, int n, bool v) {
   return r != 0;
 }
 
-// Bias of the 128 packed rows of Q tile j (-inf where no row exists).
-__device__ inline float qrow_bias(const PassArgs& p, const SeqInfo& si, int g, int j, int r) {
-  const int tok = si.q0 + j * p.tokq + r / p.G;
-  if (r < p.tokq * p.G && tok < si.len)
-    return p.bias[((size_t)g * p.T + si.start + si.q0 + (size_t)j * p.tokq) * p.G + r];
-  return -INFINITY;
-}
-
-__device__ void write_row_bias(const PassArgs& p, const SeqInfo& si, int g, int tok, int hg,
-                               float lse2) {
-  const float w = curve_weight(tok, si.len, p.a, p.b);
-  p.bias[((size_t)g * p.T + si.start + tok) * p.G + hg] = w > 0.f ? log2f(w) - lse2 : -INFINITY;
-}
-
 // Merge two (reference max, sum) pairs of the same row.
 __device__ inline float2 lse_merge(float2 x, float2 y) {
   if (!(y.y > 0.f)) return x;
   if (!(x.y > 0.f)) return y;
   const float M = fmaxf(x.x, y.x);
   return make_float2(M, x.y * ex2_approx(x.x - M) + y.y * ex2_approx(y.x - M));
+}
+
+// Bias of packed row r of Q tile j (-inf where no row exists): log2 of the
+// row's forgetting-curve weight minus log2 of its softmax normaliser, merged
+// from the pass-1 partials of the CTAs (units) that shared the row's keys,
+// in unit order.
+__device__ inline float qrow_bias(const PassArgs& p, const SeqInfo& si, int g, int j, int r) {
+  const int tok = si.q0 + j * p.tokq + r / p.G;
+  if (!(r < p.tokq * p.G && tok < si.len)) return -INFINITY;
+  const int ngrp = (si.nqt + kMaxStat1 - 1) / kMaxStat1;     // pass-1 groups per head
+  const Entry& e = p.e1[si.e1 + g * ngrp + j / kMaxStat1];
+  const float2* src = p.part1 + ((size_t)e.unit_base * kMaxStat + j % kMaxStat1) * kTile + r;
+  constexpr size_t kStride = (size_t)kMaxStat * kTile;
+  constexpr int kBatch = 8;
+  float2 acc = make_float2(-INFINITY, 0.f);
+  for (int u0 = 0; u0 < e.n_units; u0 += kBatch) {
+    float2 x[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b)
+      x[b] = u0 + b < e.n_units ? __ldcg(src + (size_t)(u0 + b) * kStride)
+                                : make_float2(-INFINITY, 0.f);
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) acc = lse_merge(acc, x[b]);
+  }
+  const float w = curve_weight(tok, si.len, p.a, p.b);
+  return w > 0.f ? log2f(w) - (acc.x + log2f(acc.y)) : -INFINITY;
 }
 
 template <int D, int PASS>
@@ -541,20 +554,23 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
     const bool fail = bar_vote_or(kBarAll, kEpiThreads, !ok || *s.abort);
     if (fail) { ok = false; continue; }
     if (PASS == 2 && e.mode == kModeP2Q) continue;
-    constexpr bool p1 = PASS == 1;
+    if (PASS == 1) {
+      // the row partials; pass 2 merges them where it reads the rows
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int i = wg + 2 * k;
+        if (i >= e.n_stat) break;
+        p.part1[((size_t)unit * kMaxStat + i) * kTile + t] = make_float2(m[k], l[k]);
+      }
+      continue;
+    }
     if (e.n_units == 1) {
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int i = wg + 2 * k;
         if (i >= e.n_stat) break;
-        if (p1) {
-          const int tok = si.q0 + (e.stat0 + i) * p.tokq + t / p.G;
-          if (t < p.tokq * p.G && tok < si.len)
-            write_row_bias(p, si, g, tok, t % p.G, m[k] + log2f(l[k]));
-        } else {
-          const int key = (e.stat0 + i) * kTile + t;
-          if (key < si.len) p.scores[(size_t)g * p.T + si.start + key] = l[k];
-        }
+        const int key = (e.stat0 + i) * kTile + t;
+        if (key < si.len) p.scores[(size_t)g * p.T + si.start + key] = l[k];
       }
       continue;
     }
@@ -562,48 +578,20 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
     for (int k = 0; k < 2; ++k) {
       const int i = wg + 2 * k;
       if (i >= e.n_stat) break;
-      const size_t slot = ((size_t)unit * kMaxStat + i) * kTile + t;
-      if (p1) p.part1[slot] = make_float2(m[k], l[k]); else p.part2[slot] = l[k];
+      p.part2[((size_t)unit * kMaxStat + i) * kTile + t] = l[k];
     }
     __threadfence();
     bar_sync(kBarAll, kEpiThreads);
-    if (tid == 0)
-      *s.last = atomicAdd(p1 ? &p.c1[ei] : &p.c2[ei], 1u) == (uint32_t)(e.n_units - 1);
+    if (tid == 0) *s.last = atomicAdd(&p.c2[ei], 1u) == (uint32_t)(e.n_units - 1);
     bar_sync(kBarAll, kEpiThreads);
     if (!*s.last) continue;
     __threadfence();
-    // each thread merges row t of the slots wg and wg + 2: the partials of all
+    // each thread merges key t of the slots wg and wg + 2: the partials of all
     // units, in unit order, up to 40 loads in flight
     constexpr size_t kStride = (size_t)kMaxStat * kTile;
     constexpr int kBatch = 20;
     const int nu = e.n_units;
-    if (p1) {
-      float2 acc[2] = {make_float2(-INFINITY, 0.f), make_float2(-INFINITY, 0.f)};
-      for (int u0 = 0; u0 < nu; u0 += kBatch) {
-        float2 x[2][kBatch];
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int i = wg + 2 * k;
-          const size_t base = ((size_t)e.unit_base * kMaxStat + i) * kTile + t;
-#pragma unroll
-          for (int b = 0; b < kBatch; ++b)
-            x[k][b] = i < e.n_stat && u0 + b < nu
-                          ? __ldcg(p.part1 + base + (size_t)(u0 + b) * kStride)
-                          : make_float2(-INFINITY, 0.f);
-        }
-#pragma unroll
-        for (int k = 0; k < 2; ++k)
-#pragma unroll
-          for (int b = 0; b < kBatch; ++b) acc[k] = lse_merge(acc[k], x[k][b]);
-      }
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int i = wg + 2 * k;
-        const int tok = si.q0 + (e.stat0 + i) * p.tokq + t / p.G;
-        if (i < e.n_stat && t < p.tokq * p.G && tok < si.len)
-          write_row_bias(p, si, g, tok, t % p.G, acc[k].x + log2f(acc[k].y));
-      }
-    } else {
+    {
       float acc[2] = {0.f, 0.f};
       for (int u0 = 0; u0 < nu; u0 += kBatch) {
         float x[2][kBatch];

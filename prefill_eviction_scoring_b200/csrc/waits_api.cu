@@ -89,7 +89,6 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   pa.seqs = reinterpret_cast<SeqInfo*>(base + L.seqs);
   pa.e1 = reinterpret_cast<Entry*>(base + L.e1);
   pa.e2 = reinterpret_cast<Entry*>(base + L.e2);
-  pa.c1 = reinterpret_cast<uint32_t*>(base + L.c1);
   pa.c2 = reinterpret_cast<uint32_t*>(base + L.c2);
   pa.max_e1 = L.max_e1;
   pa.max_e2 = L.max_e2;
@@ -115,9 +114,7 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   p.seqs = pa.seqs;
   p.e1 = pa.e1;
   p.e2 = pa.e2;
-  p.c1 = pa.c1;
   p.c2 = pa.c2;
-  p.bias = reinterpret_cast<float*>(base + L.bias);
   p.part1 = reinterpret_cast<float2*>(base + L.part1);
   p.part2 = reinterpret_cast<float*>(base + L.part2);
   p.scores = scores;

@@ -70,7 +70,7 @@ struct PlanHeader {
 
 // ------------------------------------------------------ workspace layout ---
 struct Layout {
-  size_t header, seqs, e1, e2, c1, c2, bias, part1, part2, total;
+  size_t header, seqs, e1, e2, c2, part1, part2, total;
   int64_t max_e1, max_e2, max_u1, max_u2;
 };
 
@@ -91,9 +91,7 @@ __host__ inline Layout make_layout(int64_t nseq, int64_t T, int64_t Hq, int64_t 
   L.seqs = take(sizeof(SeqInfo) * (size_t)nseq);
   L.e1 = take(sizeof(Entry) * (size_t)L.max_e1);
   L.e2 = take(sizeof(Entry) * (size_t)L.max_e2);
-  L.c1 = take(sizeof(uint32_t) * (size_t)L.max_e1);
   L.c2 = take(sizeof(uint32_t) * (size_t)L.max_e2);
-  L.bias = take(sizeof(float) * (size_t)(Hq * T));
   L.part1 = take(sizeof(float2) * (size_t)L.max_u1 * kMaxStat * kTile);
   L.part2 = take(sizeof(float) * (size_t)L.max_u2 * kMaxStat * kTile);
   L.total = off;
@@ -187,8 +185,7 @@ struct PlanArgs {
   SeqInfo* seqs;
   Entry* e1;
   Entry* e2;
-  uint32_t* c1;
-  uint32_t* c2;
+  uint32_t* c2;        // pass-2 unit counters (last-arriver merges), zeroed
   int64_t max_e1, max_e2, max_u1, max_u2;
   float* scores;  // zero-filled for sequences without active rows
 };
@@ -204,9 +201,7 @@ struct PassArgs {
   const SeqInfo* seqs;
   const Entry* e1;
   const Entry* e2;
-  uint32_t* c1;
   uint32_t* c2;
-  float* bias;         // [Hkv, T, G] log2 w - log2-sum-exp, active rows only
   float2* part1;       // [units, 4, 128] (reference max, sum) in log2 units
   float* part2;        // [units, 4, 128] partial column sums
   float* scores;       // [Hkv, T]
