@@ -43,10 +43,10 @@ KERNELS_PER_LAYER = 5   # plan, pass 1, pass 2, select, compact
 EVENT_EVERY = 8         # timed region: CUDA events around every 8th layer's scorer
 MUFU_EX2_PER_CLK_PER_SM = 16   # sm_100: 4 SFU lanes per SM sub-partition x 4
 # DRAM bytes (read + write) of one waits_score call on one llama8b layer, from
-# the ncu capture summarised in profiles/score_tc_select_llama8b_1layer.md
+# the ncu capture summarised in profiles/score_tc_select_compact_llama8b_1layer.md
 # (both scorer passes).  Valid only for the scorer source it was taken on.
-PROFILED_SCORER = {"sha256_prefix": "22a1d5293a8e63d5", "dram_bytes": 68_125_952 + 1_314_048 +
-                   68_119_552 + 1_133_312}
+PROFILED_SCORER = {"sha256_prefix": "4665f86b9a4cf283", "dram_bytes": 68_107_776 + 1_477_120 +
+                   68_406_784 + 1_191_168}
 
 
 def parse():

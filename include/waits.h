@@ -193,7 +193,7 @@ waits_status waits_compress_host(const waits_shape* shape,
 /*
  * Largest scratch waits_score_static can use: 32 MiB, enough for one
  * Llama-3.1-8B-shaped layer (N = 32768, 32/8 heads) whose
- * waits_workspace_size() is 19.2 MiB.
+ * waits_workspace_size() is 13.3 MiB.
  */
 #define WAITS_STATIC_WORKSPACE_BYTES (32u << 20)
 

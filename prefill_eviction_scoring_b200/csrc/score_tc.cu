@@ -453,8 +453,8 @@ __device__ inline float qrow_bias(const PassArgs& p, const SeqInfo& si, int g, i
   if (!(r < p.tokq * p.G && tok < si.len)) return -INFINITY;
   const int ngrp = (si.nqt + kMaxStat1 - 1) / kMaxStat1;     // pass-1 groups per head
   const Entry& e = p.e1[si.e1 + g * ngrp + j / kMaxStat1];
-  const float2* src = p.part1 + ((size_t)e.unit_base * kMaxStat + j % kMaxStat1) * kTile + r;
-  constexpr size_t kStride = (size_t)kMaxStat * kTile;
+  const float2* src = p.part1 + ((size_t)e.unit_base * kMaxStat1 + j % kMaxStat1) * kTile + r;
+  constexpr size_t kStride = (size_t)kMaxStat1 * kTile;
   constexpr int kBatch = 8;
   float2 acc = make_float2(-INFINITY, 0.f);
   for (int u0 = 0; u0 < e.n_units; u0 += kBatch) {
@@ -560,7 +560,7 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
       for (int k = 0; k < 2; ++k) {
         const int i = wg + 2 * k;
         if (i >= e.n_stat) break;
-        p.part1[((size_t)unit * kMaxStat + i) * kTile + t] = make_float2(m[k], l[k]);
+        p.part1[((size_t)unit * kMaxStat1 + i) * kTile + t] = make_float2(m[k], l[k]);
       }
       continue;
     }

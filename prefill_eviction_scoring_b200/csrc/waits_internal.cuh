@@ -92,7 +92,7 @@ __host__ inline Layout make_layout(int64_t nseq, int64_t T, int64_t Hq, int64_t 
   L.e1 = take(sizeof(Entry) * (size_t)L.max_e1);
   L.e2 = take(sizeof(Entry) * (size_t)L.max_e2);
   L.c2 = take(sizeof(uint32_t) * (size_t)L.max_e2);
-  L.part1 = take(sizeof(float2) * (size_t)L.max_u1 * kMaxStat * kTile);
+  L.part1 = take(sizeof(float2) * (size_t)L.max_u1 * kMaxStat1 * kTile);
   L.part2 = take(sizeof(float) * (size_t)L.max_u2 * kMaxStat * kTile);
   L.total = off;
   return L;
@@ -202,7 +202,7 @@ struct PassArgs {
   const Entry* e1;
   const Entry* e2;
   uint32_t* c2;
-  float2* part1;       // [units, 4, 128] (reference max, sum) in log2 units
+  float2* part1;       // [units, 2, 128] (reference max, sum) in log2 units
   float* part2;        // [units, 4, 128] partial column sums
   float* scores;       // [Hkv, T]
   uint32_t* status;
