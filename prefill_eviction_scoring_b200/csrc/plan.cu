@@ -39,6 +39,8 @@ __device__ void fill_entry_p1(int tokq, const SeqInfo& si, int s, int local, Ent
   const int last = qtile_last_token(si, e.stat0 + e.n_stat - 1, tokq);
   e.step0 = 0;
   e.n_steps = last / kTile + 1;
+  // K tiles from the one holding the group's first row on cross the diagonal
+  e.n_masked = e.n_steps - (si.q0 + e.stat0 * tokq) / kTile;
 }
 
 __device__ void fill_entry_p2(int tokq, const SeqInfo& si, int s, int local, Entry& e) {
@@ -52,6 +54,8 @@ __device__ void fill_entry_p2(int tokq, const SeqInfo& si, int s, int local, Ent
     e.n_stat = si.nqt;
     e.step0 = 0;
     e.n_steps = si.nkt;
+    // K tiles from the one holding the first active row on cross the diagonal
+    e.n_masked = e.n_steps - si.q0 / kTile;
   } else {
     e.mode = kModeP2K;
     e.stat0 = e.grp * kMaxStat;

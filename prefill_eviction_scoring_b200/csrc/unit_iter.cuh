@@ -33,9 +33,20 @@ struct UnitIter {
       const Entry& en = E[a];
       const int64_t u = cta - en.first_cta, nu = en.n_units, n = en.n_steps;
       if (u < 0 || u >= nu) return false;
+      // split the entry's cost evenly: its last n_masked steps (on the
+      // causal diagonal) cost kMaskedCost each, the others 1.  Every unit
+      // must keep a step (pass 2 reads every unit's partials), which holds
+      // when a unit's share of the cost is at least one masked step; else
+      // the steps are split evenly.
+      int64_t m = en.n_masked < 0 ? 0 : (en.n_masked > n ? n : en.n_masked);
+      if (n - m + m * kMaskedCost < nu * kMaskedCost) m = 0;
+      const int64_t plain = n - m, cost = plain + m * kMaskedCost;
+      auto step_at = [&](int64_t c) {
+        return c <= plain ? c : plain + (c - plain + kMaskedCost - 1) / kMaskedCost;
+      };
       e = a;
-      pos = en.sbase + u * n / nu;
-      hi = en.sbase + (u + 1) * n / nu;
+      pos = en.sbase + step_at(u * cost / nu);
+      hi = en.sbase + step_at((u + 1) * cost / nu);
       return pos < hi;
     }
     const int64_t lo = ((int64_t)cta * S + P - 1) / P;

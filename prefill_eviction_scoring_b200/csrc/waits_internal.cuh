@@ -54,8 +54,13 @@ struct Entry {
   int32_t unit_base; // partial-result slot of this entry's first unit
   int32_t n_units;   // CTAs (units) covering the entry
   int32_t first_cta;
-  int32_t pad[3];
+  int32_t n_masked;  // trailing steps that reach the causal diagonal (slower)
+  int32_t pad[2];
 };
+
+// Cost of a step on the causal diagonal (masked exp path) in units of an
+// unmasked step, for splitting an entry's steps evenly by time.
+constexpr int kMaskedCost = 3;   // measured: 2 and 3 alike, 1% better than 1
 
 struct PlanHeader {
   uint32_t status;     // WAITS_DEV_* bits, cleared by the planner
