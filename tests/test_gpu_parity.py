@@ -177,9 +177,11 @@ def test_host_buffer_entry_point():
     ((40000, 3000), 16, 1024, 7, False),      # ragged batch
     ((50000,), 16, 4096, 1, False),           # every score equal
     ((9000,), 0, 300, 100000, False),         # nearly distinct scores, R = 0
-    ((150000, 700), 16, 2048, 3000, False),   # pool larger than the cluster's shared memory
+    ((150000, 700), 16, 2048, 3000, False),   # pool past the cluster's staging (8 x 8192 keys)
     ((5000, 2600), 8, 512, 40, True),         # negative values, -0 and +0
     ((3000,), 16, 2999, 5, False),            # one pool position dropped
+    ((21, 40, 17, 300), 16, 20, 6, False),    # pools of a few keys: CTAs without a group
+    (tuple(range(1, 4000, 97)), 16, 64, 30, False),   # 42 sequences, N <= B among them
 ])
 def test_select_exact_on_synthetic_scores(lens, R, B, levels, signed):
     """waits_select alone, on scores with controlled ties, equals the
