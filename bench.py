@@ -39,7 +39,7 @@ METRIC = "prompt tokens/s scored+compacted per layer (8B shape, N=32K); % of roo
 UNIT = "tokens/s"
 CONFIG = "llama8b"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1590.0}
-KERNELS_PER_LAYER = 5   # plan, pass 1, pass 2, select, compact
+KERNELS_OUTSIDE_SCORE = 2   # select, compact (waits_score_kernels gives the scorer's)
 EVENT_EVERY = 8         # timed region: CUDA events around every 8th layer's scorer
 MUFU_EX2_PER_CLK_PER_SM = 16   # sm_100: 4 SFU lanes per SM sub-partition x 4
 # DRAM bytes (read + write) of one waits_score call on one llama8b layer, from
@@ -108,6 +108,14 @@ def profiled_traffic():
     with open(src, "rb") as f:
         h = hashlib.sha256(f.read()).hexdigest()
     return PROFILED_SCORER["dram_bytes"] if h.startswith(PROFILED_SCORER["sha256_prefix"]) else None
+
+
+def score_kernels(lib, shape, a, b):
+    """Kernels one waits_score call enqueues (2, or 3 with the planner)."""
+    n = ctypes.c_int32(0)
+    _lib.check("waits_score_kernels", lib.waits_score_kernels(ctypes.byref(shape), a, b,
+                                                              ctypes.byref(n)))
+    return n.value
 
 
 def peaks():
@@ -460,7 +468,7 @@ def run_ours(args):
                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                "config": config_dict(args, L, lay0.lens, wl.CONFIGS[CONFIG]),
                "roofline": roof, "roofline_other": other, "cpu_baseline": cpu, "e2e": e2e,
-               "gpu_launches": KERNELS_PER_LAYER * L * K, "clocks": clk,
+               "gpu_launches": (score_kernels(lib, shape, a, b) + KERNELS_OUTSIDE_SCORE) * L * K, "clocks": clk,
                "per_layer_us": {"score": round(t_score * 1e3, 2),
                                 "select": round(t_sel * 1e3, 2),
                                 "compact": round(t_comp * 1e3, 2)},

@@ -92,6 +92,20 @@ const char* waits_last_error(void);
 waits_status waits_workspace_size(const waits_shape* shape, size_t* bytes);
 
 /*
+ * Number of kernels one waits_score call with this shape, a and b enqueues:
+ * 2 (the two scorer passes) when every scorer CTA can rebuild the work plan
+ * itself -- at most 32 sequences and, from a bound on the rows whose fp32
+ * weight is non-zero (about b + 89/a per sequence), at most 32 planned
+ * entries per pass with all active rows of a sequence in 4 Q tiles -- else
+ * 3 (a planner kernel first).  Either way the results are the same.
+ * Host-only; touches no device state.
+ * Errors: WAITS_ERR_ARG if shape or kernels is NULL, or a < 0 / non-finite,
+ * or b < 0; shape errors as below.
+ */
+waits_status waits_score_kernels(const waits_shape* shape, float a, int32_t b,
+                                 int32_t* kernels);
+
+/*
  * Accumulative forgetting-curve score (README opening summary).  For every
  * sequence, KV head g and key k:
  *   scores[g * T + cu[i] + k] =

@@ -4,69 +4,12 @@
 // on the device keeps the whole path asynchronous (no host round trip for
 // sequence lengths).  Intermediate values stay in shared memory / registers;
 // global memory is only written.
-#include "waits_internal.cuh"
+#include "plan_core.cuh"
 
 namespace waits {
 namespace {
 
 constexpr int kSmemSeqs = 512;     // sequences kept in shared memory
-
-__device__ inline int ceil_div(int x, int y) { return (x + y - 1) / y; }
-
-// Number of stationary groups per (sequence, KV head) for each pass.
-__device__ inline int groups_p1(const SeqInfo& si) {
-  return si.len > si.q0 ? ceil_div(si.nqt, kMaxStat1) : 0;
-}
-__device__ inline int groups_p2(const SeqInfo& si) {
-  if (si.len <= si.q0) return 0;
-  return si.nqt <= kMaxStat ? 1 : ceil_div(si.nkt, kMaxStat);
-}
-
-// Last position covered by Q tile j (sequence-local).
-__device__ inline int qtile_last_token(const SeqInfo& si, int j, int tokq) {
-  const int e = si.q0 + (j + 1) * tokq;
-  return (e < si.len ? e : si.len) - 1;
-}
-
-__device__ void fill_entry_p1(int tokq, const SeqInfo& si, int s, int local, Entry& e) {
-  const int ng = groups_p1(si);
-  e.seq = s;
-  e.g = local / ng;
-  e.grp = local % ng;
-  e.mode = kModeP1;
-  e.stat0 = e.grp * kMaxStat1;
-  e.n_stat = min(kMaxStat1, si.nqt - e.stat0);
-  const int last = qtile_last_token(si, e.stat0 + e.n_stat - 1, tokq);
-  e.step0 = 0;
-  e.n_steps = last / kTile + 1;
-  // K tiles from the one holding the group's first row on cross the diagonal
-  e.n_masked = e.n_steps - (si.q0 + e.stat0 * tokq) / kTile;
-}
-
-__device__ void fill_entry_p2(int tokq, const SeqInfo& si, int s, int local, Entry& e) {
-  const int ng = groups_p2(si);
-  e.seq = s;
-  e.g = local / ng;
-  e.grp = local % ng;
-  if (si.nqt <= kMaxStat) {
-    e.mode = kModeP2Q;
-    e.stat0 = 0;
-    e.n_stat = si.nqt;
-    e.step0 = 0;
-    e.n_steps = si.nkt;
-    // K tiles from the one holding the first active row on cross the diagonal
-    e.n_masked = e.n_steps - si.q0 / kTile;
-  } else {
-    e.mode = kModeP2K;
-    e.stat0 = e.grp * kMaxStat;
-    e.n_stat = min(kMaxStat, si.nkt - e.stat0);
-    // first Q tile whose last position reaches the group's first key
-    const int x = e.stat0 * kTile - si.q0;
-    const int j0 = x > 0 ? x / tokq : 0;
-    e.step0 = j0;
-    e.n_steps = si.nqt - j0;
-  }
-}
 
 struct Seqs {
   SeqInfo* sm;   // shared copy (nseq <= kSmemSeqs) or null
@@ -110,7 +53,7 @@ __device__ void plan_pass(const Seqs& S, int nseq, int tokq, int n, int grid, En
   }
   const int64_t Stot = carry;
   const int64_t P = Stot < (int64_t)grid ? Stot : (int64_t)grid;
-  auto cta_at = [&](int64_t c) { return (c * P + Stot / 2) / Stot; };
+  auto cta_at = [&](int64_t c) { return waits::cta_at(c, P, Stot); };
   // can every entry own whole CTAs?
   bool aligned = n <= P && Stot > 0;
   {
@@ -184,15 +127,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs p) {
     SeqInfo si{};
     int64_t v1 = 0, v2 = 0;
     if (s < p.nseq) {
-      const int lo = p.cu[s], hi = p.cu[s + 1];
-      const bool bad = (s == 0 && lo != 0) || hi < lo || hi > p.T ||
-                       (hi - lo) > p.max_seqlen || (s == p.nseq - 1 && hi != p.T);
+      bool bad;
+      si = seq_info(p.cu, s, p.nseq, p.T, p.max_seqlen, p.tokq, p.a, p.b, bad);
       if (bad) atomicOr(&s_bad, 1);
-      si.start = lo;
-      si.len = bad ? 0 : hi - lo;
-      si.q0 = first_active_row(si.len, p.a, p.b);
-      si.nqt = (si.len - si.q0 + p.tokq - 1) / p.tokq;
-      si.nkt = (si.len + kTile - 1) / kTile;
       v1 = (int64_t)p.Hkv * groups_p1(si);
       v2 = (int64_t)p.Hkv * groups_p2(si);
     }

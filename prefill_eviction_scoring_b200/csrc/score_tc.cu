@@ -20,6 +20,7 @@
 // stay in a thread), so neither pass needs a cross-thread reduction.
 // Every wait is bounded; a timeout sets WAITS_DEV_TIMEOUT and the CTA exits
 // after its copies and MMAs in flight have landed.
+#include "plan_core.cuh"
 #include "sm100.cuh"
 #include "unit_iter.cuh"
 
@@ -63,7 +64,7 @@ struct Cfg {
                                     + kWGs * 2 * kTile           // streamed Q biases
                                     + 2 * kWGs * kMaxStat * kTile;  // per-WG state
   static constexpr size_t kSmem = 1024 + (size_t)(kStat + kStages) * kTileBytes +
-                                  kFloats * sizeof(float) + 256;
+                                  kFloats * sizeof(float) + sizeof(LocalPlan) + 256;
 };
 
 struct Smem {
@@ -80,6 +81,7 @@ struct Smem {
   uint64_t* tfull;
   uint64_t* tempty;
   uint64_t* done;
+  LocalPlan* lp;          // the plan, when each CTA builds it
   uint32_t* tmem_slot;
   volatile int* abort;
   int* last;
@@ -97,7 +99,8 @@ __device__ Smem carve(uint8_t* raw) {
   s.bias_strm = s.bias_stat + kMaxStat * kTile;
   s.st_m = s.bias_strm + kWGs * 2 * kTile;
   s.st_l = s.st_m + kWGs * kMaxStat * kTile;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.st_l + kWGs * kMaxStat * kTile);
+  s.lp = reinterpret_cast<LocalPlan*>(s.st_l + kWGs * kMaxStat * kTile);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.lp + 1);
   s.full = bars;
   s.empty = s.full + C::kStages;
   s.stat_full = s.empty + C::kStages;
@@ -622,14 +625,13 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
 template <int D, int PASS>
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
-                    const __grid_constant__ CUtensorMap tmK, PassArgs p) {
+                    const __grid_constant__ CUtensorMap tmK, const PassArgs pa) {
   using C = Cfg<D, PASS>;
   extern __shared__ uint8_t smem_raw[];
   const Smem s = carve<D, PASS>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr bool p1 = PASS == 1;
-  const PlanHeader* H = p.hdr;
-  const Entry* E = p1 ? p.e1 : p.e2;
+  PassArgs p = pa;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
@@ -661,6 +663,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_wait();
     pdl_allow_next();
   }
+  if (p.local_plan) {
+    // every CTA plans for itself (cu_seqlens is complete: pass 1 has waited
+    // above, and pass 2 starts only after pass 1 has)
+    if (warp == 0)
+      warp_plan(p.cu, p.nseq, p.T, p.max_seqlen, p.Hkv, p.tokq, p.a, p.b, (int)gridDim.x, !p1,
+                *s.lp);
+    __syncthreads();
+    p.hdr = &s.lp->hdr;
+    p.seqs = s.lp->seqs;
+    p.e1 = s.lp->e1;
+    p.e2 = s.lp->e2;
+    if (p1) {
+      // this call's device status word, and zero scores for sequences
+      // without an active row (the planner kernel's duties)
+      if (blockIdx.x == 0 && threadIdx.x == 0) *pa.status = s.lp->hdr.status;
+      if (s.lp->hdr.status == 0) {
+        const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+        for (int q = 0; q < p.nseq; ++q) {
+          const SeqInfo si = s.lp->seqs[q];
+          if (si.len == 0 || si.q0 < si.len) continue;
+          for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+               i < (int64_t)si.len * p.Hkv; i += stride)
+            p.scores[(i / si.len) * p.T + si.start + i % si.len] = 0.0f;
+        }
+      }
+    }
+  }
+  const PlanHeader* H = p.hdr;
+  const Entry* E = p1 ? p.e1 : p.e2;
 
   UnitIter it;
   const bool have = it.init(E, p1 ? H->n_e1 : H->n_e2, p1 ? H->s1 : H->s2,

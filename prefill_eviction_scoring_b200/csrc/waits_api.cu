@@ -4,7 +4,7 @@
 #include <cstdio>
 #include <cstring>
 
-#include "waits_internal.cuh"
+#include "plan_core.cuh"
 
 #include <cstdarg>
 
@@ -62,6 +62,25 @@ int grid_size() {
   return sms < kMaxGrid ? sms : kMaxGrid;
 }
 
+// Whether every scorer CTA can rebuild the plan itself (plan_core.cuh): at
+// most kLocalMax sequences and kLocalMax entries in each pass, and every
+// sequence's active rows within the stationary Q tiles of one pass-2 entry.
+// The bound on a sequence's active rows (those whose fp32 weight is not 0,
+// about b + 89/a of them) is loose by a few rows; the device counts exactly
+// and flags a plan overflow rather than run if the bound was ever short.
+bool local_plan_fits(const waits_shape* s, float a, int32_t b) {
+  if (s->nseq > kLocalMax) return false;
+  const int tokq = tokens_per_qtile(s->num_q_heads / s->num_kv_heads);
+  double rows = s->max_seqlen;                       // a = 0: every row is active
+  if (a > 0.0f)
+    rows = std::fmin(rows, (double)b + 8.0 + std::ceil(89.0 / a) + s->max_seqlen / 4194304.0);
+  const int64_t nqt = (int64_t)std::ceil(rows / tokq);
+  if (nqt > kMaxStat) return false;
+  const int64_t e1 = (int64_t)s->num_kv_heads * s->nseq * ((nqt + kMaxStat1 - 1) / kMaxStat1);
+  const int64_t e2 = (int64_t)s->num_kv_heads * s->nseq;
+  return e1 <= kLocalMax && e2 <= kLocalMax;
+}
+
 uint32_t* status_word(void* ws, size_t bytes) {
   if (!ws || bytes < sizeof(PlanHeader) || !aligned(ws, 256)) return nullptr;
   return &reinterpret_cast<PlanHeader*>(ws)->status;
@@ -95,8 +114,12 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   pa.max_u1 = L.max_u1;
   pa.max_u2 = L.max_u2;
   pa.scores = scores;
-  cudaError_t err = launch_plan(pa, st);
-  if (err != cudaSuccess) return cuda_fail("planner launch", err);
+  const bool local = local_plan_fits(s, a, b);
+  cudaError_t err = cudaSuccess;
+  if (!local) {
+    err = launch_plan(pa, st);
+    if (err != cudaSuccess) return cuda_fail("planner launch", err);
+  }
 
   PassArgs p{};
   p.Q = static_cast<const uint16_t*>(Q);
@@ -119,6 +142,10 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   p.part2 = reinterpret_cast<float*>(base + L.part2);
   p.scores = scores;
   p.status = &pa.hdr->status;
+  p.local_plan = local ? 1 : 0;
+  p.cu = s->cu_seqlens;
+  p.nseq = s->nseq;
+  p.max_seqlen = s->max_seqlen;
   err = launch_score_passes(p, grid, st);
   if (err != cudaSuccess) return cuda_fail("scorer launch", err);
   return WAITS_OK;
@@ -185,6 +212,15 @@ waits_status waits_workspace_size(const waits_shape* shape, size_t* bytes) {
   const waits_status st = check_shape(shape);
   if (st != WAITS_OK) return st;
   *bytes = layout_of(shape).total;
+  return WAITS_OK;
+}
+
+waits_status waits_score_kernels(const waits_shape* shape, float a, int32_t b,
+                                 int32_t* kernels) {
+  if (!kernels || !std::isfinite(a) || a < 0.0f || b < 0) return WAITS_ERR_ARG;
+  const waits_status st = check_shape(shape);
+  if (st != WAITS_OK) return st;
+  *kernels = local_plan_fits(shape, a, b) ? 2 : 3;
   return WAITS_OK;
 }
 

@@ -211,6 +211,11 @@ struct PassArgs {
   float* part2;        // [units, 4, 128] partial column sums
   float* scores;       // [Hkv, T]
   uint32_t* status;
+  // local plan: every CTA rebuilds the (small) plan in shared memory from
+  // cu_seqlens, and no planner kernel runs
+  int local_plan;
+  const int32_t* cu;
+  int nseq, max_seqlen;
 };
 
 // ------------------------------------------- programmatic dependent launch ---

@@ -139,3 +139,29 @@ def test_python_binding_fails_loudly_without_library(tmp_path):
             _lib.load(str(tmp_path / "missing.so"))
     finally:
         _lib._lib = saved
+
+
+def _kernels(lib, shape, a, b):
+    n = ctypes.c_int32(0)
+    st = lib.waits_score_kernels(ctypes.byref(shape), a, b, ctypes.byref(n))
+    return st, n.value
+
+
+def test_score_kernel_count(lib):
+    """Small plans are rebuilt inside the scorer (2 kernels); large ones take
+    the planner kernel first (3)."""
+    llama8b = _shape(total_tokens=32768, max_seqlen=32768)
+    assert _kernels(lib, llama8b, 1.0, 16) == (0, 2)     # ~105 active rows: 4 Q tiles
+    assert _kernels(lib, llama8b, 10.0, 1) == (0, 2)
+    assert _kernels(lib, llama8b, 0.0, 16) == (0, 3)     # every row active
+    assert _kernels(lib, llama8b, 0.01, 128) == (0, 3)   # ~9000 active rows
+    batch = _shape(nseq=40, total_tokens=40 * 512, max_seqlen=512, num_kv_heads=4,
+                   num_q_heads=28)
+    assert _kernels(lib, batch, 1.0, 16) == (0, 3)        # more than 32 sequences
+    two = _shape(nseq=2, total_tokens=2 * 8192, max_seqlen=8192)
+    assert _kernels(lib, two, 1.0, 16) == (0, 2)          # 8 heads x 2 x 2 = 32 pass-1 entries
+    three = _shape(nseq=3, total_tokens=3 * 8192, max_seqlen=8192)
+    assert _kernels(lib, three, 1.0, 16) == (0, 3)        # 48 pass-1 entries
+    assert _kernels(lib, llama8b, -1.0, 16)[0] == 1
+    assert _kernels(lib, llama8b, 1.0, -1)[0] == 1
+    assert lib.waits_score_kernels(ctypes.byref(llama8b), 1.0, 16, None) == 1
