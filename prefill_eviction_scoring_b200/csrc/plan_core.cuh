@@ -84,8 +84,13 @@ __device__ inline void fill_entry_p2(int tokq, const SeqInfo& si, int s, int loc
   }
 }
 
-// CTA boundary nearest to global step c when P CTAs share S steps.
-__device__ inline int64_t cta_at(int64_t c, int64_t P, int64_t S) { return (c * P + S / 2) / S; }
+// CTA boundary nearest to global step c when P CTAs share S steps (32-bit
+// arithmetic when c * P + S / 2 fits it, c <= S).
+__device__ inline int64_t cta_at(int64_t c, int64_t P, int64_t S) {
+  if (S * P + S / 2 <= 0xFFFFFFFFll)
+    return (int64_t)(((uint32_t)c * (uint32_t)P + (uint32_t)(S / 2)) / (uint32_t)S);
+  return (c * P + S / 2) / S;
+}
 
 // ------------------------------------------------------------ local plan ---
 constexpr int kLocalMax = 32;   // sequences, and entries per pass, of a local plan
@@ -133,11 +138,13 @@ __device__ inline void warp_plan_pass(const SeqInfo* seqs, int nseq, int tokq, i
   const int64_t c = warp_exclusive_scan(v, &Stot);
   const int64_t P = Stot < (int64_t)grid ? Stot : (int64_t)grid;
   bool aligned = n <= P && Stot > 0;
+  int64_t f0 = 0, f1 = 0;   // the entry's CTA boundaries under the aligned split
   if (aligned) {
     bool ok = true;
     if (i < n) {
-      const int64_t nu = cta_at(c + v, P, Stot) - cta_at(c, P, Stot);
-      ok = nu >= 1 && nu <= v;
+      f0 = cta_at(c, P, Stot);
+      f1 = cta_at(c + v, P, Stot);
+      ok = f1 - f0 >= 1 && f1 - f0 <= v;
     }
     aligned = __all_sync(0xffffffffu, ok);
   }
@@ -145,8 +152,8 @@ __device__ inline void warp_plan_pass(const SeqInfo* seqs, int nseq, int tokq, i
   if (i < n) {
     e.sbase = c;
     if (aligned) {
-      e.first_cta = (int)cta_at(c, P, Stot);
-      nu = cta_at(c + v, P, Stot) - e.first_cta;
+      e.first_cta = (int)f0;
+      nu = f1 - f0;
     } else {
       const int64_t f = c * P / Stot, l = (c + v - 1) * P / Stot;
       e.first_cta = (int)f;

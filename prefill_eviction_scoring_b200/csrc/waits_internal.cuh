@@ -120,9 +120,12 @@ __device__ inline float curve_weight(int q, int N, float a, int b) {
 __device__ inline int first_active_row(int N, float a, int b) {
   if (N <= 0) return 0;
   if (a == 0.0f) return 0;
-  auto active = [&](int q) { return curve_weight(q, N, a, b) != 0.0f; };
-  if (!active(N - 1)) return N;
   const float c = (float)N - (float)b - 0.5f;
+  // curve_weight(q) != 0 exactly when expf(t) is finite: 1 + expf(t) is then
+  // at most FLT_MAX and its IEEE reciprocal at least 2.9e-39 (no flush to
+  // zero); this test skips the division
+  auto active = [&](int q) { return expf(-a * ((float)q - c)) != INFINITY; };
+  if (!active(N - 1)) return N;
   float est = ceilf(c - 88.72284f / a);
   int q = est < 0.f ? 0 : (est > (float)(N - 1) ? N - 1 : (int)est);
   for (int step = 0; step < 8; ++step) {
