@@ -28,9 +28,12 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
   const int s = (int)(sg / (uint32_t)Hkv);
   const int g = (int)(sg - (uint32_t)s * (uint32_t)Hkv);
   uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
-  if (j < __ldg(kept_len + s)) {
-    const int lo = __ldg(cu + s), N = __ldg(cu + s + 1) - lo;
-    const int k = __ldg(idx + row);
+  // the four index loads are independent: issue them together, then the
+  // row loads (two dependent levels instead of four)
+  const int kl = __ldg(kept_len + s), lo = __ldg(cu + s), hi = __ldg(cu + s + 1);
+  const int k = __ldg(idx + row);
+  if (j < kl) {
+    const int N = hi - lo;
     if (k >= 0 && k < N) {
       const size_t src = ((size_t)(lo + k) * Hkv + g) * kCpr + c;
       kv = __ldg(K + src);
