@@ -45,8 +45,8 @@ MUFU_EX2_PER_CLK_PER_SM = 16   # sm_100: 4 SFU lanes per SM sub-partition x 4
 # DRAM bytes (read + write) of one waits_score call on one llama8b layer, from
 # the ncu capture summarised in profiles/score_tc_select_compact_llama8b_1layer.md
 # (both scorer passes).  Valid only for the scorer source it was taken on.
-PROFILED_SCORER = {"sha256_prefix": "4665f86b9a4cf283", "dram_bytes": 68_107_776 + 1_477_120 +
-                   68_406_784 + 1_191_168}
+PROFILED_SCORER = {"sha256_prefix": "f053c39490723286", "dram_bytes": 68_128_768 + 2_419_200 +
+                   68_427_008 + 1_462_528}
 
 
 def parse():
