@@ -2,6 +2,7 @@
 // on the caller's stream.  Declarations and contracts: include/waits.h.
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "plan_core.cuh"
@@ -69,6 +70,9 @@ int grid_size() {
 // about b + 89/a of them) is loose by a few rows; the device counts exactly
 // and flags a plan overflow rather than run if the bound was ever short.
 bool local_plan_fits(const waits_shape* s, float a, int32_t b) {
+  // WAITS_PLANNER_KERNEL=1 (debugging, tests): always plan with the planner kernel
+  const char* force = std::getenv("WAITS_PLANNER_KERNEL");
+  if (force && force[0] == '1') return false;
   if (s->nseq > kLocalMax) return false;
   const int tokq = tokens_per_qtile(s->num_q_heads / s->num_kv_heads);
   double rows = s->max_seqlen;                       // a = 0: every row is active

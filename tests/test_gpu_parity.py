@@ -113,6 +113,37 @@ def test_deterministic_bits():
     assert np.array_equal(a["idx"], b["idx"])
 
 
+@pytest.mark.parametrize("make,a,b", [
+    (lambda: wl.make_layer("llama8b", device="cuda"), 1.0, 16),
+    (lambda: wl.make_layer("ragged", lens=(1500, 900, 77), heads=(8, 2), device="cuda"), 1.0, 16),
+    (lambda: wl.make_layer("ragged", lens=(300,), heads=(4, 1), device="cuda"), 10.0, 1),
+])
+def test_in_cta_plan_equals_planner_kernel(make, a, b, monkeypatch):
+    """The plan every scorer CTA rebuilds for itself and the planner kernel's
+    plan give the same scores bit for bit (same units, same order)."""
+    import ctypes
+    from prefill_eviction_scoring_b200 import _lib, api
+    lay = make()
+    T, Hq, d = lay.Q.shape
+    shape = api.make_shape(lay.cu_seqlens, T, lay.max_seqlen, Hq, lay.K.shape[1], d)
+    lib = _lib.load()
+
+    def kernels():
+        n = ctypes.c_int32(0)
+        _lib.check("waits_score_kernels", lib.waits_score_kernels(ctypes.byref(shape), a, b,
+                                                                  ctypes.byref(n)))
+        return n.value
+
+    monkeypatch.delenv("WAITS_PLANNER_KERNEL", raising=False)
+    assert kernels() == 2
+    s_local = api.score(lay.Q, lay.K, lay.cu_seqlens, sigmoid_a=a, window=b).clone()
+    monkeypatch.setenv("WAITS_PLANNER_KERNEL", "1")
+    assert kernels() == 3
+    s_kernel = api.score(lay.Q, lay.K, lay.cu_seqlens, sigmoid_a=a, window=b)
+    torch.cuda.synchronize()
+    assert torch.equal(s_local.view(torch.int32), s_kernel.view(torch.int32))
+
+
 def test_separate_calls_equal_fused():
     """waits_score, waits_select and waits_compact called one by one give
     the same bits as waits_compress."""
