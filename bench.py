@@ -5,7 +5,7 @@ Workload: the Llama-3.1-8B-shaped stack -- 32 layers with independently
 seeded bf16 Q/K/V (sink + 64 heavy hitters per KV head), batch 1, N=32768,
 32 query / 8 KV heads, d=128, a=1, b=16, R=16, B=2048 (``--budget``).
 A step runs score -> select -> compact once for every layer, through the C
-ABI (waits_score, waits_select, waits_compact on one stream).
+ABI (waits_score, then waits_select_compact, on one stream).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -39,7 +39,7 @@ METRIC = "prompt tokens/s scored+compacted per layer (8B shape, N=32K); % of roo
 UNIT = "tokens/s"
 CONFIG = "llama8b"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1590.0}
-KERNELS_OUTSIDE_SCORE = 2   # select, compact (waits_score_kernels gives the scorer's)
+KERNELS_OUTSIDE_SCORE = 1   # select+compact (waits_score_kernels gives the scorer's)
 EVENT_EVERY = 8         # timed region: CUDA events around every 8th layer's scorer
 MUFU_EX2_PER_CLK_PER_SM = 16   # sm_100: 4 SFU lanes per SM sub-partition x 4
 # DRAM bytes (read + write) of one waits_score call on one llama8b layer, from
@@ -230,7 +230,7 @@ class ClockSampler:
 
 
 class LayerCall:
-    """Preallocated buffers for one layer and the three C-ABI calls."""
+    """Preallocated buffers for one layer and its C-ABI calls."""
 
     def __init__(self, lay, B, shape, workspace, ws_bytes):
         self.lay = lay
@@ -251,16 +251,11 @@ class LayerCall:
                                self.lay.K.data_ptr(), a, b, self.scores.data_ptr(),
                                self.ws.data_ptr(), self.ws_bytes, stream)
 
-    def select(self, lib, R, stream):
-        return lib.waits_select(ctypes.byref(self.shape), self.scores.data_ptr(), R, self.B,
-                                self.idx.data_ptr(), self.kept.data_ptr(), self.ws.data_ptr(),
-                                self.ws_bytes, stream)
-
-    def compact(self, lib, stream):
-        return lib.waits_compact(ctypes.byref(self.shape), self.lay.K.data_ptr(),
-                                 self.lay.V.data_ptr(), self.idx.data_ptr(), self.kept.data_ptr(),
-                                 self.B, self.Ko.data_ptr(), self.Vo.data_ptr(),
-                                 self.ws.data_ptr(), self.ws_bytes, stream)
+    def select_compact(self, lib, R, stream):
+        return lib.waits_select_compact(
+            ctypes.byref(self.shape), self.scores.data_ptr(), self.lay.K.data_ptr(),
+            self.lay.V.data_ptr(), R, self.B, self.idx.data_ptr(), self.kept.data_ptr(),
+            self.Ko.data_ptr(), self.Vo.data_ptr(), self.ws.data_ptr(), self.ws_bytes, stream)
 
 
 def cpu_oracle_sample(lay, a, b, R, B, g=0):
@@ -333,15 +328,12 @@ def run_ours(args):
             _lib.check("waits_score", c.score(lib, a, b, sp))
             if timed:
                 evs[i][1].record(stream)
-            _lib.check("waits_select", c.select(lib, R, sp))
+            _lib.check("waits_select_compact", c.select_compact(lib, R, sp))
             if evs is not None and which == "all":
                 evs[i][2].record(stream)
-            _lib.check("waits_compact", c.compact(lib, sp))
-            if evs is not None and which == "all":
-                evs[i][3].record(stream)
 
     def new_events(k):
-        return [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in calls]
+        return [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in calls]
                 for _ in range(k)]
 
     for _ in range(args.warmup):
@@ -370,7 +362,7 @@ def run_ours(args):
         t_score = D.max(statistics.mean(e[0].elapsed_time(e[1]) for s_ in evs
                                         for i, e in enumerate(s_) if i % EVENT_EVERY == 0))
 
-    # select and compact durations: a few more steps with events around
+    # select+compact duration: a few more steps with events around
     # every call (outside the timed region; they cut the overlap of calls)
     KS = min(K, 5)
     evs2 = new_events(KS)
@@ -381,14 +373,14 @@ def run_ours(args):
     D.barrier()
     if args.kernel_events != "score":
         t_score = D.max(statistics.mean(e[0].elapsed_time(e[1]) for s_ in evs2 for e in s_))
-    t_sel = D.max(statistics.mean(e[1].elapsed_time(e[2]) for s_ in evs2 for e in s_))
-    t_comp = D.max(statistics.mean(e[2].elapsed_time(e[3]) for s_ in evs2 for e in s_))
+    t_sc = D.max(statistics.mean(e[1].elapsed_time(e[2]) for s_ in evs2 for e in s_))
 
     N = lay0.max_seqlen
     tokens_per_step = D.world * L * sum(lay0.lens)
     value = tokens_per_step / (ms / 1e3)
     flops, logits = scorer_flops(lay0.lens, Hq, d, a, b)
     sel_b, comp_b = select_compact_bytes(lay0.lens, Hkv, d, B)
+    sc_b = sel_b + comp_b
     pk, pk_kind = peaks()
     peak_t = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
     achieved_t = flops / (t_score / 1e3) / 1e12
@@ -419,13 +411,10 @@ def run_ours(args):
     hbm = float(pk.get("hbm_gbs"))
     other = [
         tensor_roof,
-        {"kernel": "select", "bound": "hbm", "achieved": round(sel_b / (t_sel / 1e3) / 1e9, 1),
-         "peak": hbm, "unit": "GB/s", "frac": round(sel_b / (t_sel / 1e3) / 1e9 / hbm, 4),
-         "bytes_per_launch": sel_b, "launch_ms": round(t_sel, 4)},
-        {"kernel": "compact", "bound": "hbm",
-         "achieved": round(comp_b / (t_comp / 1e3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
-         "frac": round(comp_b / (t_comp / 1e3) / 1e9 / hbm, 4), "bytes_per_launch": comp_b,
-         "launch_ms": round(t_comp, 4)}]
+        {"kernel": "select+compact (waits_select_compact, one kernel)", "bound": "hbm",
+         "achieved": round(sc_b / (t_sc / 1e3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
+         "frac": round(sc_b / (t_sc / 1e3) / 1e9 / hbm, 4), "bytes_per_launch": sc_b,
+         "launch_ms": round(t_sc, 4)}]
 
     # ---- end to end through the host-buffer entry point
     E = min(args.e2e_layers, L)
@@ -470,8 +459,7 @@ def run_ours(args):
                "roofline": roof, "roofline_other": other, "cpu_baseline": cpu, "e2e": e2e,
                "gpu_launches": (score_kernels(lib, shape, a, b) + KERNELS_OUTSIDE_SCORE) * L * K, "clocks": clk,
                "per_layer_us": {"score": round(t_score * 1e3, 2),
-                                "select": round(t_sel * 1e3, 2),
-                                "compact": round(t_comp * 1e3, 2)},
+                                "select+compact": round(t_sc * 1e3, 2)},
                "active_logits_per_layer": logits}
         print(json.dumps(out), flush=True)
     D.close()

@@ -156,6 +156,20 @@ waits_status waits_compact(const waits_shape* shape, const void* K, const void* 
                            size_t workspace_bytes, void* stream);
 
 /*
+ * waits_select followed by waits_compact, in one kernel: the same idx,
+ * kept_len, K_out and V_out bit for bit.  The selecting CTAs copy the K and
+ * V rows of the positions they keep as soon as those positions are known, so
+ * the compaction costs no launch or wait of its own.  (waits_compress uses
+ * it.)  Arguments as in the two calls; the indices come from the selection,
+ * so WAITS_DEV_BAD_INDEX cannot arise.
+ * Errors: ARG, SHAPE, UNSUPPORTED, CUDA.
+ */
+waits_status waits_select_compact(const waits_shape* shape, const float* scores,
+                                  const void* K, const void* V, int32_t R, int32_t B,
+                                  int32_t* idx, int32_t* kept_len, void* K_out, void* V_out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * score -> select -> compact in one call, all enqueued on `stream`.
  * Arguments as above; `scores` is an output too.
  */

@@ -8,5 +8,6 @@ it is missing (there is no fallback).
 
 from .api import (  # noqa: F401
     Compressor, HostCompressor, compact, compress, score, score_static, select,
+    select_compact,
     workspace_bytes, make_shape)
 from ._lib import WaitsError, WaitsLibraryError  # noqa: F401

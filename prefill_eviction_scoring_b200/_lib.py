@@ -70,6 +70,7 @@ SIGNATURES = {
                                       ctypes.POINTER(ctypes.c_uint32)]),
     "waits_score_static": (_I, [_PSHAPE, _P, _P, _F, _I, _P, _P]),
     "waits_score_kernels": (_I, [_PSHAPE, _F, _I, ctypes.POINTER(ctypes.c_int32)]),
+    "waits_select_compact": (_I, [_PSHAPE, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 STATIC_WORKSPACE_BYTES = 32 << 20   # WAITS_STATIC_WORKSPACE_BYTES

@@ -190,6 +190,32 @@ def compact(K: torch.Tensor, V: torch.Tensor, cu_seqlens: torch.Tensor, idx: tor
     return Ko, Vo
 
 
+def select_compact(scores: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                   cu_seqlens: torch.Tensor, *, recent_budget: int, budget: int,
+                   max_seqlen: Optional[int] = None
+                   ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
+    """``(idx, kept_len, K_out, V_out)``: ``select`` then ``compact`` in one
+    kernel (``waits_select_compact``)."""
+    _need_cuda("scores", scores, torch.float32)
+    _need_cuda("K", K, torch.bfloat16)
+    _need_cuda("V", V, torch.bfloat16)
+    _need_cuda("cu_seqlens", cu_seqlens, torch.int32)
+    lib = _lib.load()
+    T, Hkv, d = K.shape
+    nseq = cu_seqlens.numel() - 1
+    B = int(budget)
+    shape = make_shape(cu_seqlens, T, _max_seqlen(cu_seqlens, max_seqlen), Hkv, Hkv, d)
+    idx = torch.empty((nseq, Hkv, B), dtype=torch.int32, device=K.device)
+    kept = torch.empty((nseq,), dtype=torch.int32, device=K.device)
+    Ko = torch.empty((nseq, Hkv, B, d), dtype=torch.bfloat16, device=K.device)
+    Vo = torch.empty_like(Ko)
+    st = lib.waits_select_compact(ctypes.byref(shape), _ptr(scores), _ptr(K), _ptr(V),
+                                  int(recent_budget), B, _ptr(idx), _ptr(kept), _ptr(Ko),
+                                  _ptr(Vo), None, 0, _stream(K.device))
+    _lib.check("waits_select_compact", st)
+    return idx, kept, Ko, Vo
+
+
 def compress(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, *,
              sigmoid_a: float, window: int, recent_budget: int, budget: int,
              max_seqlen: Optional[int] = None):

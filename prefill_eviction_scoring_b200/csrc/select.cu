@@ -20,6 +20,12 @@
 // and places its kept positions with block scans, ties to tau taken lowest
 // index first.  The first pass stages the slice's images in shared memory,
 // so the later passes read no global memory.
+//
+// With the KV copy (waits_select_compact, waits_compress) the same kernel
+// also compacts K and V: after each output round the CTA copies the rows of
+// the slots it has just filled (a contiguous range of slots, their source
+// positions staged in shared memory), and the CTAs of the cluster share the
+// recent window's rows and any zero rows.
 #include "waits_internal.cuh"
 
 namespace waits {
@@ -32,6 +38,8 @@ constexpr int kBins1 = 4096;                     // bits 20..31
 constexpr int kCopies = 4;                       // local first-digit histograms (warp % 4)
 constexpr int kBins2 = 1024;                     // bits 10..19, then 0..9
 constexpr int kMaxPer = kBins1 / kSelThreads;    // bins per thread in find_bin
+constexpr int kOutGroups = 2;                    // output pass: groups per thread and round
+constexpr int kRoundKeys = 4 * kOutGroups * kSelThreads;   // positions per output round
 
 // Monotone map of fp32 to uint32: a < b (as floats, -0 == +0) iff
 // key(a) < key(b).  Scores from waits_score are >= 0, but waits_select takes
@@ -52,7 +60,42 @@ struct SelSmem {
   int64_t scan[32];
   uint32_t digit;                    // find_bin's result
   int32_t above;
+  int32_t src[kRoundKeys];           // KV copy: source position of each slot of a round
 };
+
+// K / V of the compaction (null K: selection only).  Rows are d / 8 16-byte
+// vectors (1 << log_cpr).
+struct KVCopy {
+  const uint4* K;
+  const uint4* V;
+  uint4* Ko;
+  uint4* Vo;
+  int log_cpr;
+};
+
+// Output rows [r0, r1) of (sequence s, KV head g): slot j gets source
+// position src_of(j) of the sequence (starting at token lo), or zeros when
+// src_of(j) < 0.  All threads of the CTA, one 16-byte vector each in turn.
+template <typename F>
+__device__ inline void copy_rows(const KVCopy& c, int Hkv, int B, int s, int g, int lo, int r0,
+                                 int r1, F src_of) {
+  const int cpr = 1 << c.log_cpr;
+  const int n = (r1 - r0) << c.log_cpr;
+  const size_t out0 = ((size_t)s * Hkv + g) * (size_t)B;
+  for (int v = (int)threadIdx.x; v < n; v += blockDim.x) {
+    const int j = r0 + (v >> c.log_cpr), col = v & (cpr - 1);
+    const int src = src_of(j);
+    const size_t dst = ((out0 + j) << c.log_cpr) + col;
+    if (src >= 0) {
+      const size_t from = ((((size_t)lo + src) * Hkv + g) << c.log_cpr) + col;
+      c.Ko[dst] = __ldg(c.K + from);
+      c.Vo[dst] = __ldg(c.V + from);
+    } else {
+      c.Ko[dst] = make_uint4(0, 0, 0, 0);
+      c.Vo[dst] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
 
 // ---------------------------------------------------------- cluster ops ---
 __device__ inline uint32_t cluster_rank() {
@@ -145,10 +188,11 @@ __device__ void find_bin(SelSmem& sm, const uint32_t* h, int nb, int need) {
   __syncthreads();
 }
 
+template <bool COPY>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const float* __restrict__ scores, const int32_t* __restrict__ cu, int nseq, int T,
     int Hkv, int R, int B, int32_t* __restrict__ idx, int32_t* __restrict__ kept_len,
-    uint32_t* status) {
+    uint32_t* status, KVCopy kv) {
   extern __shared__ uint4 dyn_smem[];
   uint4* stage = dyn_smem;                                     // [kStageGroups]
   SelSmem& sm = *reinterpret_cast<SelSmem*>(dyn_smem + kStageGroups);
@@ -170,6 +214,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   const int lo = cu[s], hi = cu[s + 1];
   int32_t* out = idx + ((size_t)s * Hkv + g) * B;
   const bool bad = (s == 0 && lo != 0) || hi < lo || hi > T || (s == nseq - 1 && hi != T);
+  // the cluster's share of output rows [0, n): rank r takes [n r / kC, n (r + 1) / kC)
+  auto share = [&](int n, int& r0, int& r1) {
+    r0 = (int)((int64_t)n * rank / kC);
+    r1 = (int)((int64_t)n * (rank + 1) / kC);
+  };
   if (bad) {
     if (rank == 0) {
       for (int j = tid; j < B; j += kSelThreads) out[j] = -1;
@@ -178,6 +227,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
         if (status) atomicOr(status, WAITS_DEV_BAD_SEQLENS);
       }
     }
+    if (COPY) {
+      int r0, r1;
+      share(B, r0, r1);
+      copy_rows(kv, Hkv, B, s, g, 0, r0, r1, [](int) { return -1; });
+    }
     return;
   }
   const int N = hi - lo;
@@ -185,12 +239,23 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   if (N <= B) {
     if (rank == 0)
       for (int j = tid; j < B; j += kSelThreads) out[j] = j < N ? j : -1;
+    if (COPY) {
+      int r0, r1;
+      share(B, r0, r1);
+      copy_rows(kv, Hkv, B, s, g, lo, r0, r1, [N](int j) { return j < N ? j : -1; });
+    }
     return;
   }
   const int want = B - R;            // positions taken from the pool by score
   const int pool = N - R;            // > want because N > B
   if (rank == 0)
     for (int j = tid; j < R; j += kSelThreads) out[want + j] = pool + j;   // recent window
+  if (COPY) {
+    int r0, r1;
+    share(R, r0, r1);
+    copy_rows(kv, Hkv, B, s, g, lo, want + r0, want + r1,
+              [want, pool](int j) { return pool + (j - want); });
+  }
   if (want == 0) return;
 
   const float* sc = scores + (size_t)g * T + lo;
@@ -344,8 +409,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 
   // ---- ascending positions: rounds of kOutGroups * kSelThreads consecutive
   // groups (kOutGroups per thread), one block scan of packed (above tau,
-  // equal to tau) counts per round
-  constexpr int kOutGroups = 2;
+  // equal to tau) counts per round; the kept positions of a round fill a
+  // contiguous range of slots
   for (int i0 = g_lo; i0 < g_hi; i0 += kOutGroups * kSelThreads) {
     const int ib = i0 + kOutGroups * tid;
     uint32_t gtm = 0, eqm = 0;     // bit 4j + e: position 4(ib + j) + e - off
@@ -367,6 +432,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     int64_t tot;
     const int64_t ex = block_exclusive_scan(mine, &tot, sm.scan);
     const int64_t gt_before = gt_base + (ex >> 32), eq_before = eq_base + (ex & 0xFFFFFFFFll);
+    // this round's slots: [slot0, slot0 + kept)
+    const int64_t slot0 = gt_base + (eq_base < need ? eq_base : (int64_t)need);
     const int p0 = 4 * ib - P.off;
     uint32_t any = gtm | eqm;
     while (any) {
@@ -377,11 +444,22 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
       const bool gt = (gtm >> b) & 1u;
       if (gt || eb < need) {
         const int64_t pos = gb + (eb < need ? eb : (int64_t)need);
-        if (pos < want) out[pos] = p0 + b;
+        if (pos < want) {
+          out[pos] = p0 + b;
+          if (COPY) sm.src[pos - slot0] = p0 + b;
+        }
       }
     }
     gt_base += tot >> 32;
     eq_base += tot & 0xFFFFFFFFll;
+    if (COPY) {
+      const int64_t slot1 = gt_base + (eq_base < need ? eq_base : (int64_t)need);
+      __syncthreads();
+      copy_rows(kv, Hkv, B, s, g, lo, (int)slot0, (int)(slot1 < want ? slot1 : want),
+                [&](int j) { return sm.src[j - slot0]; });
+      // the next round's scan (block barriers) orders these reads of sm.src
+      // before its writes
+    }
   }
 }
 
@@ -389,16 +467,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 
 cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int T, int Hkv,
                           int R, int B, int32_t* idx, int32_t* kept_len, uint32_t* status,
-                          cudaStream_t s) {
+                          cudaStream_t s, const uint16_t* K, const uint16_t* V, int d,
+                          uint16_t* Ko, uint16_t* Vo) {
   const int64_t grid = (int64_t)nseq * Hkv * kC;
   if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
   const int dyn = kStageGroups * (int)sizeof(uint4) + (int)sizeof(SelSmem);
-  cudaError_t err = cudaFuncSetAttribute(select_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+  KVCopy kv{reinterpret_cast<const uint4*>(K), reinterpret_cast<const uint4*>(V),
+            reinterpret_cast<uint4*>(Ko), reinterpret_cast<uint4*>(Vo), d == 128 ? 4 : 3};
+  auto kernel = K ? select_kernel<true> : select_kernel<false>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
   if (err != cudaSuccess) return err;
-  return launch_pdl_cluster(select_kernel, dim3((unsigned)grid), dim3(kSelThreads), kC,
-                            (size_t)dyn, s, scores, cu, nseq, T, Hkv, R, B, idx, kept_len,
-                            status);
+  return launch_pdl_cluster(kernel, dim3((unsigned)grid), dim3(kSelThreads), kC, (size_t)dyn, s,
+                            scores, cu, nseq, T, Hkv, R, B, idx, kept_len, status, kv);
 }
 
 }  // namespace waits

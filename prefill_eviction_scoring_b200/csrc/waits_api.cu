@@ -281,15 +281,29 @@ waits_status waits_compress(const waits_shape* shape, const void* Q, const void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = enqueue_score(shape, Q, K, a, b, scores, workspace, s);
   if (st != WAITS_OK) return st;
-  uint32_t* status = status_word(workspace, workspace_bytes);
-  cudaError_t err = launch_select(scores, shape->cu_seqlens, shape->nseq, shape->total_tokens,
-                                  shape->num_kv_heads, R, B, idx, kept_len, status, s);
-  if (err != cudaSuccess) return cuda_fail("select launch", err);
-  err = launch_compact(static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
-                       shape->cu_seqlens, idx, kept_len, shape->nseq, shape->num_kv_heads,
-                       shape->head_dim, B, static_cast<uint16_t*>(K_out),
-                       static_cast<uint16_t*>(V_out), status, s);
-  if (err != cudaSuccess) return cuda_fail("compact launch", err);
+  const cudaError_t err = launch_select(
+      scores, shape->cu_seqlens, shape->nseq, shape->total_tokens, shape->num_kv_heads, R, B,
+      idx, kept_len, status_word(workspace, workspace_bytes), s, static_cast<const uint16_t*>(K),
+      static_cast<const uint16_t*>(V), shape->head_dim, static_cast<uint16_t*>(K_out),
+      static_cast<uint16_t*>(V_out));
+  if (err != cudaSuccess) return cuda_fail("select-compact launch", err);
+  return WAITS_OK;
+}
+
+waits_status waits_select_compact(const waits_shape* shape, const float* scores,
+                                  const void* K, const void* V, int32_t R, int32_t B,
+                                  int32_t* idx, int32_t* kept_len, void* K_out, void* V_out,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  waits_status st = check_shape(shape);
+  if (st == WAITS_OK) st = check_select_args(scores, R, B, idx, kept_len);
+  if (st == WAITS_OK) st = check_compact_args(K, V, idx, kept_len, B, K_out, V_out);
+  if (st != WAITS_OK) return st;
+  const cudaError_t err = launch_select(
+      scores, shape->cu_seqlens, shape->nseq, shape->total_tokens, shape->num_kv_heads, R, B,
+      idx, kept_len, status_word(workspace, workspace_bytes), static_cast<cudaStream_t>(stream),
+      static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V), shape->head_dim,
+      static_cast<uint16_t*>(K_out), static_cast<uint16_t*>(V_out));
+  if (err != cudaSuccess) return cuda_fail("select-compact launch", err);
   return WAITS_OK;
 }
 

@@ -276,9 +276,13 @@ void set_error_detail(const char* fmt, ...);
 // Host-side launchers (one per translation unit).
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
 cudaError_t launch_score_passes(const PassArgs& a, int grid, cudaStream_t s);
+// K == nullptr: selection only; else also the compaction of K and V into
+// Ko, Vo (the rows of the kept positions, zeros past kept_len).
 cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int T,
                           int Hkv, int R, int B, int32_t* idx, int32_t* kept_len,
-                          uint32_t* status, cudaStream_t s);
+                          uint32_t* status, cudaStream_t s, const uint16_t* K = nullptr,
+                          const uint16_t* V = nullptr, int d = 0, uint16_t* Ko = nullptr,
+                          uint16_t* Vo = nullptr);
 cudaError_t launch_compact(const uint16_t* K, const uint16_t* V, const int32_t* cu,
                            const int32_t* idx, const int32_t* kept_len, int nseq,
                            int Hkv, int d, int B, uint16_t* Ko, uint16_t* Vo,

@@ -232,3 +232,73 @@ def test_select_exact_on_synthetic_scores(lens, R, B, levels, signed):
     ref_idx, ref_kept = oracle.select(s.double().cpu().numpy(), cu.cpu().numpy(), R, B)
     np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
     np.testing.assert_array_equal(kept.cpu().numpy(), ref_kept)
+
+
+_SELECT_COMPACT_CASES = [
+    ((20000,), 64, 2048, 50, 128),            # many ties at the threshold
+    ((40000, 3000), 16, 1024, 7, 64),         # ragged batch
+    ((50000,), 16, 4096, 1, 128),             # every score equal: one run of slots
+    ((9000,), 0, 300, 100000, 128),           # R = 0
+    ((150000, 700), 16, 2048, 3000, 128),     # pool past the cluster's staging
+    ((3000,), 16, 2999, 5, 64),               # one pool position dropped
+    ((3000,), 3000, 3000, 5, 128),            # want = 0: the recent window only
+    ((21, 40, 17, 300), 16, 20, 6, 128),      # pools of a few keys, N <= B among them
+    (tuple(range(1, 4000, 97)), 16, 64, 30, 64),   # 42 sequences
+    ((70000,), 16, 9000, 2, 128),             # rounds of 4096 slots, the last one partial
+]
+
+
+@pytest.mark.parametrize("lens,R,B,levels,d", _SELECT_COMPACT_CASES)
+def test_select_compact_exact(lens, R, B, levels, d):
+    """waits_select_compact (selection and the K/V copy in one kernel) equals
+    the oracle's selection and compaction, bit for bit, and the two separate
+    calls."""
+    from prefill_eviction_scoring_b200 import api
+    g = torch.Generator(device="cuda")
+    g.manual_seed(321)
+    Hkv, T = 2, sum(lens)
+    s = torch.randint(0, levels, (Hkv, T), generator=g, device="cuda").float() / 64.0
+    K = torch.randint(-32768, 32767, (T, Hkv, d), generator=g, device="cuda",
+                      dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    V = torch.randint(-32768, 32767, (T, Hkv, d), generator=g, device="cuda",
+                      dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device="cuda")
+    idx, kept, Ko, Vo = api.select_compact(s, K, V, cu, recent_budget=R, budget=B)
+    idx2, kept2 = api.select(s, cu, recent_budget=R, budget=B)
+    Ko2, Vo2 = api.compact(K, V, cu, idx2, kept2)
+    torch.cuda.synchronize()
+    ref_idx, ref_kept = oracle.select(s.double().cpu().numpy(), cu.cpu().numpy(), R, B)
+    Kb, Vb = (t.view(torch.int16).cpu().numpy() for t in (K, V))
+    ref_K, ref_V = oracle.compact(Kb, Vb, cu.cpu().numpy(), ref_idx, ref_kept, B)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_array_equal(kept.cpu().numpy(), ref_kept)
+    np.testing.assert_array_equal(Ko.view(torch.int16).cpu().numpy(), ref_K)
+    np.testing.assert_array_equal(Vo.view(torch.int16).cpu().numpy(), ref_V)
+    assert torch.equal(idx, idx2) and torch.equal(kept, kept2)
+    assert torch.equal(Ko.view(torch.int16), Ko2.view(torch.int16))
+    assert torch.equal(Vo.view(torch.int16), Vo2.view(torch.int16))
+
+
+def test_select_compact_bad_seqlens_zero_rows():
+    """Malformed offsets: status bit set, every output row zero, no K/V read."""
+    from prefill_eviction_scoring_b200 import api, _lib
+    K = torch.ones((500, 2, 128), dtype=torch.bfloat16, device="cuda")
+    s = torch.ones((2, 500), dtype=torch.float32, device="cuda")
+    bad = torch.tensor([0, 350, 499], dtype=torch.int32, device="cuda")   # last != T
+    lib = _lib.load()
+    shape = api.make_shape(bad, 500, 350, 2, 2, 128)
+    idx = torch.empty((2, 2, 64), dtype=torch.int32, device="cuda")
+    kept = torch.empty((2,), dtype=torch.int32, device="cuda")
+    Ko = torch.full((2, 2, 64, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    Vo = torch.full_like(Ko, 7.0)
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    import ctypes
+    st = lib.waits_select_compact(ctypes.byref(shape), s.data_ptr(), K.data_ptr(), K.data_ptr(),
+                                  16, 64, idx.data_ptr(), kept.data_ptr(), Ko.data_ptr(),
+                                  Vo.data_ptr(), ws.data_ptr(), ws.numel(),
+                                  torch.cuda.current_stream().cuda_stream)
+    _lib.check("waits_select_compact", st)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) & _lib.DEV_BAD_SEQLENS
+    assert torch.all(Ko[1] == 0) and torch.all(Vo[1] == 0)
+    assert int(kept[1].item()) == 0
