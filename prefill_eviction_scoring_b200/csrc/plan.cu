@@ -199,4 +199,73 @@ cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s) {
   return launch_pdl(plan_kernel, dim3(1), dim3(threads), 0, s, a);
 }
 
+namespace {
+
+// One pass of the one-sequence plan: warp_plan_pass's rule, entry by entry.
+template <bool P1>
+void host_plan_pass(const SeqInfo& si, int tokq, int n, int grid, Entry* out, int64_t* steps,
+                    int* units, int* ctas, int* aligned_out) {
+  int64_t c[kHostPlanMax], v[kHostPlanMax], f0[kHostPlanMax], f1[kHostPlanMax];
+  int64_t S = 0;
+  for (int i = 0; i < n; ++i) {
+    out[i] = Entry{};
+    if (P1) fill_entry_p1(tokq, si, 0, i, out[i]);
+    else fill_entry_p2(tokq, si, 0, i, out[i]);
+    v[i] = out[i].n_steps;
+    c[i] = S;
+    S += v[i];
+  }
+  const int64_t P = S < (int64_t)grid ? S : (int64_t)grid;
+  bool aligned = n <= P && S > 0;
+  for (int i = 0; aligned && i < n; ++i) {
+    f0[i] = cta_at(c[i], P, S);
+    f1[i] = cta_at(c[i] + v[i], P, S);
+    aligned = f1[i] - f0[i] >= 1 && f1[i] - f0[i] <= v[i];
+  }
+  int64_t U = 0;
+  for (int i = 0; i < n; ++i) {
+    Entry& e = out[i];
+    int64_t nu;
+    e.sbase = c[i];
+    if (aligned) {
+      e.first_cta = (int)f0[i];
+      nu = f1[i] - f0[i];
+    } else {
+      const int64_t f = c[i] * P / S, l = (c[i] + v[i] - 1) * P / S;
+      e.first_cta = (int)f;
+      nu = l - f + 1;
+    }
+    e.n_units = (int)nu;
+    e.unit_base = aligned ? e.first_cta : (int)U;
+    U += nu;
+  }
+  *steps = S;
+  *units = (int)U;
+  *ctas = (int)P;
+  *aligned_out = aligned ? 1 : 0;
+}
+
+}  // namespace
+
+bool host_plan_single(int T, int max_seqlen, int Hkv, int tokq, float a, int b, int grid,
+                      HostPlan* hp) {
+  bool bad = false;
+  SeqInfo si = seq_info(0, T, 0, 1, T, max_seqlen, tokq, a, b, bad);
+  if (bad) return false;
+  const int64_t n1 = (int64_t)Hkv * groups_p1(si), n2 = (int64_t)Hkv * groups_p2(si);
+  if (n1 > kHostPlanMax || n2 > kHostPlanMax) return false;
+  if (si.len > si.q0 && si.nqt > kMaxStat) return false;   // would need stationary K tiles
+  si.e1 = 0;
+  si.e2 = 0;
+  *hp = HostPlan{};
+  hp->seq = si;
+  PlanHeader& H = hp->hdr;
+  H.status = 0u;
+  H.n_e1 = (int)n1;
+  H.n_e2 = (int)n2;
+  host_plan_pass<true>(si, tokq, (int)n1, grid, hp->e1, &H.s1, &H.n_u1, &H.p1, &H.aligned1);
+  host_plan_pass<false>(si, tokq, (int)n2, grid, hp->e2, &H.s2, &H.n_u2, &H.p2, &H.aligned2);
+  return true;
+}
+
 }  // namespace waits

@@ -10,30 +10,29 @@
 
 namespace waits {
 
-__device__ inline int ceil_div(int x, int y) { return (x + y - 1) / y; }
+__host__ __device__ inline int ceil_div(int x, int y) { return (x + y - 1) / y; }
 
 // Number of stationary groups per (sequence, KV head) for each pass.
-__device__ inline int groups_p1(const SeqInfo& si) {
+__host__ __device__ inline int groups_p1(const SeqInfo& si) {
   return si.len > si.q0 ? ceil_div(si.nqt, kMaxStat1) : 0;
 }
-__device__ inline int groups_p2(const SeqInfo& si) {
+__host__ __device__ inline int groups_p2(const SeqInfo& si) {
   if (si.len <= si.q0) return 0;
   return si.nqt <= kMaxStat ? 1 : ceil_div(si.nkt, kMaxStat);
 }
 
 // Last position covered by Q tile j (sequence-local).
-__device__ inline int qtile_last_token(const SeqInfo& si, int j, int tokq) {
+__host__ __device__ inline int qtile_last_token(const SeqInfo& si, int j, int tokq) {
   const int e = si.q0 + (j + 1) * tokq;
   return (e < si.len ? e : si.len) - 1;
 }
 
-// Sequence s: offsets, validity, first row with non-zero fp32 weight and
-// tile counts (entry offsets e1 / e2 are left to the caller).  Invalid
-// offsets give an empty sequence and set `bad`.
-__device__ inline SeqInfo seq_info(const int32_t* cu, int s, int nseq, int T, int max_seqlen,
-                                   int tokq, float a, int b, bool& bad) {
+// Sequence s with offsets [lo, hi): validity, first row with non-zero fp32
+// weight and tile counts (entry offsets e1 / e2 are left to the caller).
+// Invalid offsets give an empty sequence and set `bad`.
+__host__ __device__ inline SeqInfo seq_info(int lo, int hi, int s, int nseq, int T,
+                                            int max_seqlen, int tokq, float a, int b, bool& bad) {
   SeqInfo si{};
-  const int lo = cu[s], hi = cu[s + 1];
   bad = (s == 0 && lo != 0) || hi < lo || hi > T || (hi - lo) > max_seqlen ||
         (s == nseq - 1 && hi != T);
   si.start = lo;
@@ -44,7 +43,13 @@ __device__ inline SeqInfo seq_info(const int32_t* cu, int s, int nseq, int T, in
   return si;
 }
 
-__device__ inline void fill_entry_p1(int tokq, const SeqInfo& si, int s, int local, Entry& e) {
+// The same, reading the offsets of sequence s from cu_seqlens.
+__device__ inline SeqInfo seq_info(const int32_t* cu, int s, int nseq, int T, int max_seqlen,
+                                   int tokq, float a, int b, bool& bad) {
+  return seq_info(cu[s], cu[s + 1], s, nseq, T, max_seqlen, tokq, a, b, bad);
+}
+
+__host__ __device__ inline void fill_entry_p1(int tokq, const SeqInfo& si, int s, int local, Entry& e) {
   const int ng = groups_p1(si);
   e.seq = s;
   e.g = local / ng;
@@ -59,7 +64,7 @@ __device__ inline void fill_entry_p1(int tokq, const SeqInfo& si, int s, int loc
   e.n_masked = e.n_steps - (si.q0 + e.stat0 * tokq) / kTile;
 }
 
-__device__ inline void fill_entry_p2(int tokq, const SeqInfo& si, int s, int local, Entry& e) {
+__host__ __device__ inline void fill_entry_p2(int tokq, const SeqInfo& si, int s, int local, Entry& e) {
   const int ng = groups_p2(si);
   e.seq = s;
   e.g = local / ng;
@@ -86,7 +91,7 @@ __device__ inline void fill_entry_p2(int tokq, const SeqInfo& si, int s, int loc
 
 // CTA boundary nearest to global step c when P CTAs share S steps (32-bit
 // arithmetic when c * P + S / 2 fits it, c <= S).
-__device__ inline int64_t cta_at(int64_t c, int64_t P, int64_t S) {
+__host__ __device__ inline int64_t cta_at(int64_t c, int64_t P, int64_t S) {
   if (S * P + S / 2 <= 0xFFFFFFFFll)
     return (int64_t)(((uint32_t)c * (uint32_t)P + (uint32_t)(S / 2)) / (uint32_t)S);
   return (c * P + S / 2) / S;
@@ -101,6 +106,26 @@ struct LocalPlan {
   Entry e2[kLocalMax];
   PlanHeader hdr;
 };
+
+// ------------------------------------------------------------- host plan ---
+// A batch of one sequence can only be valid as cu_seqlens = {0, T}, so its
+// plan follows from the call's scalars: the host builds it (the same rules
+// as warp_plan with both passes) and hands it to the scorer as a kernel
+// parameter; each CTA copies it and checks cu_seqlens instead of planning.
+constexpr int kHostPlanMax = 24;   // entries per pass (keeps the parameter under 4 KB)
+
+struct __align__(16) HostPlan {
+  PlanHeader hdr;
+  SeqInfo seq;
+  Entry e1[kHostPlanMax];
+  Entry e2[kHostPlanMax];
+};
+
+// Builds the plan of the batch {0, T}; false (nothing built) when the
+// device must plan instead: an invalid or empty batch, more entries than
+// kHostPlanMax, or a pass-2 entry with stationary K tiles.
+bool host_plan_single(int T, int max_seqlen, int Hkv, int tokq, float a, int b, int grid,
+                      HostPlan* hp);
 
 __device__ inline int64_t warp_exclusive_scan(int64_t v, int64_t* total) {
   const int lane = threadIdx.x & 31;

@@ -447,30 +447,60 @@ __device__ inline float2 lse_merge(float2 x, float2 y) {
   return make_float2(M, x.y * ex2_approx(x.x - M) + y.y * ex2_approx(y.x - M));
 }
 
-// Bias of packed row r of Q tile j (-inf where no row exists): log2 of the
-// row's forgetting-curve weight minus log2 of its softmax normaliser, merged
-// from the pass-1 partials of the CTAs (units) that shared the row's keys,
-// in unit order.
-__device__ inline float qrow_bias(const PassArgs& p, const SeqInfo& si, int g, int j, int r) {
-  const int tok = si.q0 + j * p.tokq + r / p.G;
-  if (!(r < p.tokq * p.G && tok < si.len)) return -INFINITY;
-  const int ngrp = (si.nqt + kMaxStat1 - 1) / kMaxStat1;     // pass-1 groups per head
-  const Entry& e = p.e1[si.e1 + g * ngrp + j / kMaxStat1];
-  const float2* src = p.part1 + ((size_t)e.unit_base * kMaxStat1 + j % kMaxStat1) * kTile + r;
+// Bias of packed row r of the Q tiles j[k] (j[k] < 0: none; -inf where no
+// row exists): log2 of the row's curve weight minus its log2-sum-exp over
+// the keys, from the pass-1 partials of the row's units.  The partials of
+// all NR rows are loaded together (kMergeBatch units per row in flight) and
+// merged in unit order as a maximum, then a sum of the rescaled partial sums.
+template <int NR>
+__device__ inline void qrow_bias(const PassArgs& p, const SeqInfo& si, int g, const int (&j)[NR],
+                                 int r, float (&out)[NR]) {
   constexpr size_t kStride = (size_t)kMaxStat1 * kTile;
-  constexpr int kBatch = 8;
-  float2 acc = make_float2(-INFINITY, 0.f);
-  for (int u0 = 0; u0 < e.n_units; u0 += kBatch) {
-    float2 x[kBatch];
+  constexpr int kMergeBatch = 16;
+  const int ngrp = (si.nqt + kMaxStat1 - 1) / kMaxStat1;     // pass-1 groups per head
+  const float2* src[NR];
+  int nu[NR], tok[NR], numax = 0;
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b)
-      x[b] = u0 + b < e.n_units ? __ldcg(src + (size_t)(u0 + b) * kStride)
-                                : make_float2(-INFINITY, 0.f);
-#pragma unroll
-    for (int b = 0; b < kBatch; ++b) acc = lse_merge(acc, x[b]);
+  for (int k = 0; k < NR; ++k) {
+    tok[k] = si.q0 + j[k] * p.tokq + r / p.G;
+    nu[k] = 0;
+    src[k] = p.part1;
+    if (j[k] >= 0 && r < p.tokq * p.G && tok[k] < si.len) {
+      const Entry& e = p.e1[si.e1 + g * ngrp + j[k] / kMaxStat1];
+      src[k] = p.part1 + ((size_t)e.unit_base * kMaxStat1 + j[k] % kMaxStat1) * kTile + r;
+      nu[k] = e.n_units;
+    }
+    numax = max(numax, nu[k]);
   }
-  const float w = curve_weight(tok, si.len, p.a, p.b);
-  return w > 0.f ? log2f(w) - (acc.x + log2f(acc.y)) : -INFINITY;
+  float2 acc[NR];
+#pragma unroll
+  for (int k = 0; k < NR; ++k) acc[k] = make_float2(-INFINITY, 0.f);
+  for (int u0 = 0; u0 < numax; u0 += kMergeBatch) {
+    float2 x[NR][kMergeBatch];
+#pragma unroll
+    for (int k = 0; k < NR; ++k)
+#pragma unroll
+      for (int b = 0; b < kMergeBatch; ++b)
+        x[k][b] = u0 + b < nu[k] ? __ldcg(src[k] + (size_t)(u0 + b) * kStride)
+                                 : make_float2(-INFINITY, 0.f);
+#pragma unroll
+    for (int k = 0; k < NR; ++k) {
+      float M = acc[k].x;
+#pragma unroll
+      for (int b = 0; b < kMergeBatch; ++b)
+        if (x[k][b].y > 0.f) M = fmaxf(M, x[k][b].x);
+      float L = acc[k].y > 0.f ? acc[k].y * ex2_approx(acc[k].x - M) : 0.f;
+#pragma unroll
+      for (int b = 0; b < kMergeBatch; ++b)
+        if (x[k][b].y > 0.f) L += x[k][b].y * ex2_approx(x[k][b].x - M);
+      acc[k] = make_float2(M, L);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    const float w = nu[k] > 0 ? curve_weight(tok[k], si.len, p.a, p.b) : 0.f;
+    out[k] = w > 0.f ? log2f(w) - (acc[k].x + log2f(acc[k].y)) : -INFINITY;
+  }
 }
 
 template <int D, int PASS>
@@ -492,8 +522,15 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};   // P1 row state / P2K sums
     bar_sync(kBarAll, kEpiThreads);   // the previous unit's shared data is no longer read
     if (PASS == 2 && e.mode == kModeP2Q) {
-      for (int i = wg; i < e.n_stat; i += kWGs)
-        s.bias_stat[i * kTile + t] = qrow_bias(p, si, g, e.stat0 + i, t);
+      static_assert(kMaxStat == 2 * kWGs, "two stationary slots per warpgroup");
+      int js[2];
+      float bs[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) js[k] = wg + kWGs * k < e.n_stat ? e.stat0 + wg + kWGs * k : -1;
+      qrow_bias<2>(p, si, g, js, t, bs);
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (js[k] >= 0) s.bias_stat[(wg + kWGs * k) * kTile + t] = bs[k];
       bar_sync(kBarAll, kEpiThreads);
     }
     for (int st = st0; st < st1; ++st) {
@@ -502,7 +539,12 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
       ++sstep;
       float* bias_o = s.bias_strm + sb * kTile;
       if (PASS == 2 && e.mode == kModeP2K) {
-        if (wg == 0) bias_o[t] = qrow_bias(p, si, g, o, t);
+        if (wg == 0) {
+          const int js[1] = {o};
+          float bs[1];
+          qrow_bias<1>(p, si, g, js, t, bs);
+          bias_o[t] = bs[0];
+        }
         bar_sync(kBarAll, kEpiThreads);
       }
       float col = 0.f;
@@ -625,7 +667,8 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
 template <int D, int PASS>
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
-                    const __grid_constant__ CUtensorMap tmK, const PassArgs pa) {
+                    const __grid_constant__ CUtensorMap tmK, const PassArgs pa,
+                    const __grid_constant__ HostPlan hp) {
   using C = Cfg<D, PASS>;
   extern __shared__ uint8_t smem_raw[];
   const Smem s = carve<D, PASS>(smem_raw);
@@ -665,10 +708,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (p.local_plan) {
     // every CTA plans for itself (cu_seqlens is complete: pass 1 has waited
-    // above, and pass 2 starts only after pass 1 has)
-    if (warp == 0)
+    // above, and pass 2 starts only after pass 1 has), or copies the plan
+    // the host built for the batch {0, T} once cu_seqlens reads so
+    if (p.host_plan) {
+      const bool valid = p.cu[0] == 0 && p.cu[1] == p.T;   // the same two words in every thread
+      const int n1 = valid ? hp.hdr.n_e1 : 0, n2 = valid ? hp.hdr.n_e2 : 0;
+      constexpr int kVecs = (int)(sizeof(Entry) / sizeof(uint4));
+      const uint4* h1 = reinterpret_cast<const uint4*>(hp.e1);
+      const uint4* h2 = reinterpret_cast<const uint4*>(hp.e2);
+      uint4* d1 = reinterpret_cast<uint4*>(s.lp->e1);
+      uint4* d2 = reinterpret_cast<uint4*>(s.lp->e2);
+      for (int i = threadIdx.x; i < (n1 + n2) * kVecs; i += blockDim.x) {
+        if (i < n1 * kVecs) d1[i] = h1[i];
+        else d2[i - n1 * kVecs] = h2[i - n1 * kVecs];
+      }
+      if (threadIdx.x == 0) {
+        s.lp->seqs[0] = hp.seq;
+        PlanHeader h = hp.hdr;
+        if (!valid) {
+          h = PlanHeader{};
+          h.status = WAITS_DEV_BAD_SEQLENS;
+        }
+        s.lp->hdr = h;
+      }
+    } else if (warp == 0) {
       warp_plan(p.cu, p.nseq, p.T, p.max_seqlen, p.Hkv, p.tokq, p.a, p.b, (int)gridDim.x, !p1,
                 *s.lp);
+    }
     __syncthreads();
     p.hdr = &s.lp->hdr;
     p.seqs = s.lp->seqs;
@@ -755,8 +821,11 @@ bool make_map(CUtensorMap* m, const void* base, int T, int heads, int d, int box
          CUDA_SUCCESS;
 }
 
+static_assert(sizeof(HostPlan) + 2 * sizeof(CUtensorMap) + sizeof(PassArgs) + 64 <= 4096,
+              "scorer parameters must stay within 4 KB");
+
 template <int D>
-cudaError_t launch_d(const PassArgs& a, int grid, cudaStream_t st) {
+cudaError_t launch_d(const PassArgs& a, const HostPlan& hp, int grid, cudaStream_t st) {
   CUtensorMap mq, mk;
   if (!make_map(&mq, a.Q, a.T, a.Hq, D, a.G, a.tokq) ||
       !make_map(&mk, a.K, a.T, a.Hkv, D, 1, kTile))
@@ -771,7 +840,7 @@ cudaError_t launch_d(const PassArgs& a, int grid, cudaStream_t st) {
           cudaSuccess)
     return err;
   if ((err = launch_pdl(score_tc_kernel<D, 1>, dim3(grid), dim3(kThreads), smem1, st, mq, mk,
-                        a)) != cudaSuccess) {
+                        a, hp)) != cudaSuccess) {
     cudaFuncAttributes fa{};
     cudaFuncGetAttributes(&fa, score_tc_kernel<D, 1>);
     int dev = 0, optin = 0, regs = 0;
@@ -784,13 +853,16 @@ cudaError_t launch_d(const PassArgs& a, int grid, cudaStream_t st) {
                      smem1, optin, regs, kThreads);
     return err;
   }
-  return launch_pdl(score_tc_kernel<D, 2>, dim3(grid), dim3(kThreads), smem2, st, mq, mk, a);
+  return launch_pdl(score_tc_kernel<D, 2>, dim3(grid), dim3(kThreads), smem2, st, mq, mk, a,
+                    hp);
 }
 
 }  // namespace
 
-cudaError_t launch_score_passes(const PassArgs& a, int grid, cudaStream_t s) {
-  return a.d == 64 ? launch_d<64>(a, grid, s) : launch_d<128>(a, grid, s);
+cudaError_t launch_score_passes(const PassArgs& a, const HostPlan* hp, int grid, cudaStream_t s) {
+  static const HostPlan kNone{};
+  const HostPlan& h = hp ? *hp : kNone;
+  return a.d == 64 ? launch_d<64>(a, h, grid, s) : launch_d<128>(a, h, grid, s);
 }
 
 }  // namespace waits

@@ -75,24 +75,47 @@ struct KVCopy {
 
 // Output rows [r0, r1) of (sequence s, KV head g): slot j gets source
 // position src_of(j) of the sequence (starting at token lo), or zeros when
-// src_of(j) < 0.  All threads of the CTA, one 16-byte vector each in turn.
+// src_of(j) < 0.  All threads of the CTA, one 16-byte vector of K and of V
+// each per turn, kCopyUnroll turns with their loads in flight before the
+// stores.
 template <typename F>
 __device__ inline void copy_rows(const KVCopy& c, int Hkv, int B, int s, int g, int lo, int r0,
                                  int r1, F src_of) {
+  constexpr int kCopyUnroll = 4;
+  const uint4* __restrict__ K = c.K;
+  const uint4* __restrict__ V = c.V;
+  uint4* __restrict__ Ko = c.Ko;
+  uint4* __restrict__ Vo = c.Vo;
   const int cpr = 1 << c.log_cpr;
   const int n = (r1 - r0) << c.log_cpr;
+  const int nt = (int)blockDim.x;
   const size_t out0 = ((size_t)s * Hkv + g) * (size_t)B;
-  for (int v = (int)threadIdx.x; v < n; v += blockDim.x) {
-    const int j = r0 + (v >> c.log_cpr), col = v & (cpr - 1);
-    const int src = src_of(j);
-    const size_t dst = ((out0 + j) << c.log_cpr) + col;
-    if (src >= 0) {
-      const size_t from = ((((size_t)lo + src) * Hkv + g) << c.log_cpr) + col;
-      c.Ko[dst] = __ldg(c.K + from);
-      c.Vo[dst] = __ldg(c.V + from);
-    } else {
-      c.Ko[dst] = make_uint4(0, 0, 0, 0);
-      c.Vo[dst] = make_uint4(0, 0, 0, 0);
+  for (int v0 = (int)threadIdx.x; v0 < n; v0 += kCopyUnroll * nt) {
+    uint4 kx[kCopyUnroll], vx[kCopyUnroll];
+    size_t dst[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const int v = v0 + u * nt;
+      kx[u] = make_uint4(0, 0, 0, 0);
+      vx[u] = kx[u];
+      dst[u] = 0;
+      if (v < n) {
+        const int j = r0 + (v >> c.log_cpr), col = v & (cpr - 1);
+        const int src = src_of(j);
+        dst[u] = ((out0 + j) << c.log_cpr) + col;
+        if (src >= 0) {
+          const size_t from = ((((size_t)lo + src) * Hkv + g) << c.log_cpr) + col;
+          kx[u] = __ldg(K + from);
+          vx[u] = __ldg(V + from);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      if (v0 + u * nt < n) {
+        Ko[dst[u]] = kx[u];
+        Vo[dst[u]] = vx[u];
+      }
     }
   }
 }

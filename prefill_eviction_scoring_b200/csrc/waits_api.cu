@@ -69,6 +69,13 @@ int grid_size() {
 // The bound on a sequence's active rows (those whose fp32 weight is not 0,
 // about b + 89/a of them) is loose by a few rows; the device counts exactly
 // and flags a plan overflow rather than run if the bound was ever short.
+// WAITS_DEVICE_PLAN=1 (debugging, tests): a one-sequence batch is planned
+// on the device like any other instead of by the host.
+bool host_plan_allowed() {
+  const char* force = std::getenv("WAITS_DEVICE_PLAN");
+  return !(force && force[0] == '1');
+}
+
 bool local_plan_fits(const waits_shape* s, float a, int32_t b) {
   // WAITS_PLANNER_KERNEL=1 (debugging, tests): always plan with the planner kernel
   const char* force = std::getenv("WAITS_PLANNER_KERNEL");
@@ -150,7 +157,12 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   p.cu = s->cu_seqlens;
   p.nseq = s->nseq;
   p.max_seqlen = s->max_seqlen;
-  err = launch_score_passes(p, grid, st);
+  HostPlan hp;
+  p.host_plan = local && s->nseq == 1 && host_plan_allowed() &&
+                        host_plan_single(p.T, p.max_seqlen, p.Hkv, p.tokq, a, b, grid, &hp)
+                    ? 1
+                    : 0;
+  err = launch_score_passes(p, p.host_plan ? &hp : nullptr, grid, st);
   if (err != cudaSuccess) return cuda_fail("scorer launch", err);
   return WAITS_OK;
 }

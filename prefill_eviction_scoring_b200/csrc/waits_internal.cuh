@@ -3,6 +3,7 @@
 // forgetting-curve weight, and small block-level helpers.
 #pragma once
 
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 #include <utility>
@@ -117,7 +118,7 @@ __device__ inline float curve_weight(int q, int N, float a, int b) {
 // overflows), so the search starts from that estimate and walks to the
 // exact boundary, falling back to bisection if the walk is long; a = 0
 // weights every row by 1/2.
-__device__ inline int first_active_row(int N, float a, int b) {
+__host__ __device__ inline int first_active_row(int N, float a, int b) {
   if (N <= 0) return 0;
   if (a == 0.0f) return 0;
   const float c = (float)N - (float)b - 0.5f;
@@ -215,8 +216,10 @@ struct PassArgs {
   float* scores;       // [Hkv, T]
   uint32_t* status;
   // local plan: every CTA rebuilds the (small) plan in shared memory from
-  // cu_seqlens, and no planner kernel runs
+  // cu_seqlens, and no planner kernel runs; with host_plan it copies the
+  // plan the host built (one sequence) and only checks cu_seqlens
   int local_plan;
+  int host_plan;
   const int32_t* cu;
   int nseq, max_seqlen;
 };
@@ -275,7 +278,9 @@ void set_error_detail(const char* fmt, ...);
 
 // Host-side launchers (one per translation unit).
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
-cudaError_t launch_score_passes(const PassArgs& a, int grid, cudaStream_t s);
+struct HostPlan;
+// hp: the host-built plan when a.host_plan (else unused, may be null).
+cudaError_t launch_score_passes(const PassArgs& a, const HostPlan* hp, int grid, cudaStream_t s);
 // K == nullptr: selection only; else also the compaction of K and V into
 // Ko, Vo (the rows of the kept positions, zeros past kept_len).
 cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int T,

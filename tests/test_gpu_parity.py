@@ -115,6 +115,9 @@ def test_deterministic_bits():
 
 @pytest.mark.parametrize("make,a,b", [
     (lambda: wl.make_layer("llama8b", device="cuda"), 1.0, 16),
+    (lambda: wl.make_layer("llama1b", device="cuda"), 10.0, 1),
+    (lambda: wl.make_layer("ragged", lens=(5000,), heads=(14, 2), device="cuda"), 10.0, 16),
+    (lambda: wl.make_layer("ragged", lens=(40,), heads=(4, 4), device="cuda"), 1.0, 16),
     (lambda: wl.make_layer("ragged", lens=(1500, 900, 77), heads=(8, 2), device="cuda"), 1.0, 16),
     (lambda: wl.make_layer("ragged", lens=(300,), heads=(4, 1), device="cuda"), 10.0, 1),
 ])
@@ -135,12 +138,17 @@ def test_in_cta_plan_equals_planner_kernel(make, a, b, monkeypatch):
         return n.value
 
     monkeypatch.delenv("WAITS_PLANNER_KERNEL", raising=False)
+    monkeypatch.delenv("WAITS_DEVICE_PLAN", raising=False)
     assert kernels() == 2
+    # one-sequence batches: the plan the host builds, then the CTAs' own
     s_local = api.score(lay.Q, lay.K, lay.cu_seqlens, sigmoid_a=a, window=b).clone()
+    monkeypatch.setenv("WAITS_DEVICE_PLAN", "1")
+    s_device = api.score(lay.Q, lay.K, lay.cu_seqlens, sigmoid_a=a, window=b).clone()
     monkeypatch.setenv("WAITS_PLANNER_KERNEL", "1")
     assert kernels() == 3
     s_kernel = api.score(lay.Q, lay.K, lay.cu_seqlens, sigmoid_a=a, window=b)
     torch.cuda.synchronize()
+    assert torch.equal(s_local.view(torch.int32), s_device.view(torch.int32))
     assert torch.equal(s_local.view(torch.int32), s_kernel.view(torch.int32))
 
 
@@ -170,6 +178,21 @@ def test_bad_seqlens_flagged_not_faulting():
     c(lay.Q, lay.K, lay.V, 1.0, 16, 16)
     torch.cuda.synchronize()
     assert c.device_status() & _lib.DEV_BAD_SEQLENS
+
+
+@pytest.mark.parametrize("end", [499, 501])
+def test_bad_seqlens_one_sequence(end):
+    """A one-sequence batch whose offsets are not {0, T} (the host-built plan
+    is checked on the device): status bit set, no work, scores untouched."""
+    from prefill_eviction_scoring_b200 import Compressor, _lib
+    lay = wl.random_layer((500,), 8, 2, 128, seed=11, device="cuda")
+    bad = torch.tensor([0, end], dtype=torch.int32, device="cuda")
+    c = Compressor(bad, 500, 500, 8, 2, 128, 64)
+    c.scores.fill_(-7.0)
+    c(lay.Q, lay.K, lay.V, 1.0, 16, 16)
+    torch.cuda.synchronize()
+    assert c.device_status() & _lib.DEV_BAD_SEQLENS
+    assert torch.all(c.scores == -7.0)
 
 
 def test_compact_bad_index_flagged():
