@@ -129,7 +129,7 @@ __device__ inline void pair_tiles(const Entry& e, int o, int i, int& j, int& kt)
 template <int D, int PASS>
 __device__ void load_tile(const CUtensorMap* tmQ, const CUtensorMap* tmK, uint8_t* dst,
                           uint64_t* bar, const PassArgs& p, const SeqInfo& si, int g, bool is_q,
-                          int idx) {
+                          int idx, uint64_t k_policy) {
   using C = Cfg<D, PASS>;
 #pragma unroll
   for (int sb = 0; sb < C::kSub; ++sb) {
@@ -137,7 +137,8 @@ __device__ void load_tile(const CUtensorMap* tmQ, const CUtensorMap* tmK, uint8_
       tma_load_3d(dst + sb * C::kSubBytes, tmQ, bar, sb * 64, g * p.G,
                   si.start + si.q0 + idx * p.tokq);
     else
-      tma_load_3d(dst + sb * C::kSubBytes, tmK, bar, sb * 64, g, si.start + idx * kTile);
+      tma_load_3d_hint(dst + sb * C::kSubBytes, tmK, bar, sb * 64, g, si.start + idx * kTile,
+                       k_policy);
   }
 }
 
@@ -147,6 +148,10 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const P
   using C = Cfg<D, PASS>;
   const uint32_t q_bytes = (uint32_t)(D * 2 * p.G * p.tokq);
   const uint32_t k_bytes = (uint32_t)(D * 2 * kTile);
+  // K tiles stream through L2 once per pass (each CTA reads its own keys):
+  // evict them first, so that they do not push out the lines every layer
+  // reuses (Q tiles shared by CTAs, row partials, the kernels' code)
+  const uint64_t k_policy = l2_policy_evict_first();
   int stage = 0;
   uint32_t sph = 0, uph = 0;
   int issued[C::kStages];
@@ -163,15 +168,15 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const P
     mbar_arrive_expect_tx(s.stat_full, (sq ? q_bytes : k_bytes) * (uint32_t)e.n_stat);
     for (int i = 0; i < e.n_stat; ++i)
       load_tile<D, PASS>(tmQ, tmK, s.stat + i * C::kTileBytes, s.stat_full, p, si, e.g, sq,
-                   e.stat0 + i);
+                         e.stat0 + i, k_policy);
     stat_issued = 1;
     stat_ph = uph;
     uph ^= 1u;
     for (int st = st0; st < st1; ++st) {
       if (!mbar_wait(&s.empty[stage], sph ^ 1u, s.abort, p.status, kWaitLimitNs)) goto out;
       mbar_arrive_expect_tx(&s.full[stage], sq ? k_bytes : q_bytes);
-      load_tile<D, PASS>(tmQ, tmK, s.strm + stage * C::kTileBytes, &s.full[stage], p, si, e.g, !sq,
-                   e.step0 + st);
+      load_tile<D, PASS>(tmQ, tmK, s.strm + stage * C::kTileBytes, &s.full[stage], p, si, e.g,
+                         !sq, e.step0 + st, k_policy);
       issued[stage] = 1;
       issued_ph[stage] = sph;
       if (++stage == C::kStages) { stage = 0; sph ^= 1u; }

@@ -88,6 +88,17 @@ __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* a
 }
 
 // ------------------------------------------------------------------ TMA ---
+// 3-D tiled TMA load with an L2 cache policy.
+__device__ inline void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                        int y, int z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z),
+      "l"(policy)
+      : "memory");
+}
+
 __device__ inline void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
                                    int y, int z) {
   asm volatile(

@@ -104,6 +104,16 @@ __host__ inline Layout make_layout(int64_t nseq, int64_t T, int64_t Hq, int64_t 
   return L;
 }
 
+// ---------------------------------------------------------- L2 policies ---
+// Policy under which lines are the first to be evicted from L2: for data
+// that streams through once (or twice) per call, so that it does not push
+// out what every call reuses.
+__device__ inline uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // ------------------------------------------------------------ the curve ---
 // fp32 forgetting-curve weight (WAITS README, opening summary):
 // w = 1 / (1 + exp(-a (q - (N - b - 0.5)))), IEEE division, no flush to zero.
