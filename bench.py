@@ -45,8 +45,8 @@ MUFU_EX2_PER_CLK_PER_SM = 16   # sm_100: 4 SFU lanes per SM sub-partition x 4
 # DRAM bytes (read + write) of one waits_score call on one llama8b layer, from
 # the ncu capture summarised in profiles/score_tc_select_compact_llama8b_1layer.md
 # (both scorer passes).  Valid only for the scorer source it was taken on.
-PROFILED_SCORER = {"sha256_prefix": "f053c39490723286", "dram_bytes": 68_128_768 + 2_419_200 +
-                   68_427_008 + 1_462_528}
+PROFILED_SCORER = {"sha256_prefix": "c4dc12a0abdeda18", "dram_bytes": 68_140_032 + 1_554_176 +
+                   68_432_640 + 1_249_536}
 
 
 def parse():
