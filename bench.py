@@ -434,7 +434,8 @@ def run_ours(args):
     e2e_ms = D.max(t0.elapsed_time(t1)) / args.e2e_steps
     e2e = {"value": D.world * E * sum(lay0.lens) / (e2e_ms / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": hc.h2d_bytes * E, "d2h_bytes_per_step": hc.d2h_bytes * E,
-           "step": f"{E} layers through waits_compress_host (pinned host buffers)",
+           "step": f"{E} layers through waits_compress_host (pinned host buffers; "
+                   "the kept V rows are read in place over the bus)",
            "ms_per_step": round(e2e_ms, 3)}
 
     cpu = None

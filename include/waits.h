@@ -198,14 +198,21 @@ typedef struct waits_device_buffers {
  * idx, kept_len, K_out and V_out back to HOST memory, all on `stream`.
  * Only the rows the scorer can read are sent: each sequence's query rows
  * from a conservative lower bound of the first non-zero-weight row on, and
- * all of K and V.  The call returns once the copies are enqueued; the host
- * outputs are valid after the stream is synchronised.
+ * all of K.  V is read only where a row is kept: when V_host is page-locked
+ * and mapped into the device's address space (cudaHostAlloc, cudaMallocHost
+ * and cudaHostRegister memory under unified addressing, torch's
+ * pin_memory), the compaction kernel reads the kept rows straight from it
+ * over the bus and dev->V is not used; otherwise all of V is copied to
+ * dev->V first.  The call returns once the work is enqueued; the host
+ * outputs are valid after the stream is synchronised, and V_host must stay
+ * unchanged until then.
  *   cu_seqlens_host  HOST int32 [nseq + 1]
  *   Q_host, K_host, V_host, idx_host, kept_len_host, K_out_host,
  *   V_out_host       HOST, same layouts as the device versions
  *   dev              device staging buffers; dev->cu_seqlens receives the
  *                    offsets and shape->cu_seqlens is ignored
- *   h2d_bytes, d2h_bytes  optional HOST out: bytes copied each way
+ *   h2d_bytes, d2h_bytes  optional HOST out: bytes moved each way (the
+ *                    kept V rows read over the bus count as host to device)
  * Errors: as waits_compress, plus SHAPE if cu_seqlens_host is inconsistent.
  */
 waits_status waits_compress_host(const waits_shape* shape,

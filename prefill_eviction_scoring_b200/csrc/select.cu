@@ -77,13 +77,15 @@ struct KVCopy {
 // position src_of(j) of the sequence (starting at token lo), or zeros when
 // src_of(j) < 0.  All threads of the CTA, one 16-byte vector of K and of V
 // each per turn, kCopyUnroll turns with their loads in flight before the
-// stores.
+// stores.  V may be page-locked host memory mapped into the device's address
+// space (the host-buffer entry point), so it is read with plain coherent
+// loads.
 template <typename F>
 __device__ inline void copy_rows(const KVCopy& c, int Hkv, int B, int s, int g, int lo, int r0,
                                  int r1, F src_of) {
   constexpr int kCopyUnroll = 4;
   const uint4* __restrict__ K = c.K;
-  const uint4* __restrict__ V = c.V;
+  const uint4* V = c.V;
   uint4* __restrict__ Ko = c.Ko;
   uint4* __restrict__ Vo = c.Vo;
   const int cpr = 1 << c.log_cpr;
@@ -106,7 +108,7 @@ __device__ inline void copy_rows(const KVCopy& c, int Hkv, int B, int s, int g, 
         if (src >= 0) {
           const size_t from = ((((size_t)lo + src) * Hkv + g) << c.log_cpr) + col;
           kx[u] = __ldg(K + from);
-          vx[u] = __ldg(V + from);
+          vx[u] = ld_global_v4(V + from);
         }
       }
     }

@@ -375,9 +375,26 @@ waits_status waits_compress_host(const waits_shape* shape, const int32_t* cu_hos
                            static_cast<const uint8_t*>(Q_host) + off, (size_t)(N - q_lo) * qrow);
   }
   ok = ok && h2d(dev->K, K_host, (size_t)sh.total_tokens * krow);
-  ok = ok && h2d(dev->V, V_host, (size_t)sh.total_tokens * krow);
+  // V: only the kept rows are ever read.  Page-locked host memory mapped
+  // into the device's address space is read in place by the compaction
+  // (min(B, N) rows per sequence and KV head cross the bus); anything else
+  // is copied whole first.
+  const void* V_src = dev->V;
+  cudaPointerAttributes attr{};
+  if (cudaPointerGetAttributes(&attr, V_host) == cudaSuccess &&
+      attr.type == cudaMemoryTypeHost && attr.devicePointer != nullptr &&
+      aligned(attr.devicePointer, 16)) {
+    V_src = attr.devicePointer;
+    for (int i = 0; i < sh.nseq; ++i) {
+      const int N = cu_host[i + 1] - cu_host[i];
+      up += (size_t)(N < B ? N : B) * krow;
+    }
+  } else {
+    cudaGetLastError();   // an unregistered pointer is not an error here
+    ok = ok && h2d(dev->V, V_host, (size_t)sh.total_tokens * krow);
+  }
   if (!ok) return WAITS_ERR_CUDA;
-  st = waits_compress(&sh, dev->Q, dev->K, dev->V, a, b, R, B, dev->scores, dev->idx,
+  st = waits_compress(&sh, dev->Q, dev->K, V_src, a, b, R, B, dev->scores, dev->idx,
                       dev->kept_len, dev->K_out, dev->V_out, workspace, workspace_bytes, stream);
   if (st != WAITS_OK) return st;
   const size_t nidx = (size_t)sh.nseq * sh.num_kv_heads * B;

@@ -114,6 +114,16 @@ __device__ inline uint64_t l2_policy_evict_first() {
   return pol;
 }
 
+// 16-byte load through the coherent path (plain ld.global, no read-only
+// cache): valid for device memory and for mapped page-locked host memory.
+__device__ inline uint4 ld_global_v4(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 // ------------------------------------------------------------ the curve ---
 // fp32 forgetting-curve weight (WAITS README, opening summary):
 // w = 1 / (1 + exp(-a (q - (N - b - 0.5)))), IEEE division, no flush to zero.

@@ -209,21 +209,27 @@ def test_compact_bad_index_flagged():
     assert torch.equal(Ko[0, 0], lay.K[:16, 0])
 
 
-def test_host_buffer_entry_point():
-    """waits_compress_host gives the same result as the device entry point."""
+@pytest.mark.parametrize("pinned_v", [True, False])
+def test_host_buffer_entry_point(pinned_v):
+    """waits_compress_host gives the same result as the device entry point,
+    whether V is read in place (page-locked) or copied first (pageable)."""
     from prefill_eviction_scoring_b200 import HostCompressor
     lay = wl.make_layer("ragged", lens=(900, 333), heads=(14, 2), device="cuda")
     gpu = run_gpu(lay, 1.0, 16, 16, 128, canary=False)
     hc = HostCompressor(lay.cu_seqlens.cpu(), 14, 2, 128, 128)
-    Qh, Kh, Vh = (t.cpu().pin_memory() for t in (lay.Q, lay.K, lay.V))
+    Qh, Kh = (t.cpu().pin_memory() for t in (lay.Q, lay.K))
+    Vh = lay.V.cpu().pin_memory() if pinned_v else lay.V.cpu()
     Ko, Vo, idx, kept = hc(Qh, Kh, Vh, 1.0, 16, 16)
     torch.cuda.synchronize()
     assert np.array_equal(idx.numpy(), gpu["idx"])
     assert np.array_equal(Ko.view(torch.int16).numpy(), gpu["Ko"])
     assert np.array_equal(Vo.view(torch.int16).numpy(), gpu["Vo"])
-    kv = 1233 * 2 * 128 * 2 * 2
+    row = 2 * 128 * 2                           # one position of K or V, both KV heads
+    k_bytes = 1233 * row
+    v_bytes = (128 + 128) * row if pinned_v else 1233 * row   # kept rows only, or all of V
     q_active = 2 * 120 * 14 * 128 * 2          # ~b + 90/a rows per sequence
-    assert kv < hc.h2d_bytes < kv + q_active + 4096   # only the active Q rows
+    lo = k_bytes + v_bytes
+    assert lo < hc.h2d_bytes < lo + q_active + 4096   # only the active Q rows
 
 
 @pytest.mark.parametrize("lens,R,B,levels,signed", [
