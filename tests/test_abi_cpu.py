@@ -112,6 +112,29 @@ def test_select_compact_compress_errors(lib):
                               FAKE, FAKE, FAKE, FAKE, 0x200000, 10, None) == 4
 
 
+def test_select_compact_argument_errors(lib):
+    """waits_select_compact validates like waits_select and waits_compact
+    together, on the host, before any launch."""
+    sh = _shape()
+    call = lambda scores=FAKE, K=FAKE, V=FAKE, R=16, B=128, idx=FAKE, kept=FAKE, Ko=FAKE, \
+        Vo=FAKE: lib.waits_select_compact(ctypes.byref(sh), scores, K, V, R, B, idx, kept, Ko,
+                                          Vo, None, 0, None)
+    assert call(scores=None) == 1
+    assert call(R=17, B=16) == 1                    # R > B
+    assert call(R=-1) == 1
+    assert call(B=0) == 1
+    assert call(idx=None) == 1
+    assert call(kept=None) == 1
+    assert call(K=None) == 1
+    assert call(V=None) == 1
+    assert call(Ko=None) == 1
+    assert call(Vo=None) == 1
+    assert call(V=FAKE + 4) == 1                    # K/V rows must be 16-byte aligned
+    bad = _shape(nseq=0)
+    assert lib.waits_select_compact(ctypes.byref(bad), FAKE, FAKE, FAKE, 16, 128, FAKE, FAKE,
+                                    FAKE, FAKE, None, 0, None) == 2
+
+
 def test_host_variant_validates_offsets(lib):
     sh = _shape(nseq=2, total_tokens=100, max_seqlen=60)
     _, n = _ws(lib, sh)
