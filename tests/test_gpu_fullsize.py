@@ -83,3 +83,28 @@ def test_long_full_properties():
     self_idx, self_kept = oracle.select(s, cu, spec.recent, B)
     np.testing.assert_array_equal(gpu["idx"], self_idx)
     assert_compaction(lay, gpu, B)
+
+
+def test_llama8b_dense_properties():
+    """The 8B layer with a = 0 (every row active, w = 1/2: the stress shape
+    whose plan needs the planner kernel and pass 2's stationary K tiles):
+    identities that hold at any size, and the selection of the GPU's own
+    scores."""
+    spec = wl.CONFIGS["llama8b"]
+    lay = wl.make_layer("llama8b", device="cuda")
+    B = 2048
+    gpu = run_gpu(lay, 0.0, 16, spec.recent, B)
+    s = gpu["scores"]
+    N = lay.total_tokens
+    G = lay.Q.shape[1] // lay.K.shape[1]
+    assert np.all(s >= 0.0) and np.all(np.isfinite(s))
+    for g in range(s.shape[0]):
+        # every row of P sums to 1 and w = 1/2: the scores of a head sum to G N / 2
+        assert abs(s[g].astype(np.float64).sum() - G * N / 2) <= 1e-4 * G * N / 2
+        # the last key is seen by the last row only
+        assert s[g, N - 1] <= G * 0.5 * (1 + 1e-5)
+    cu = lay.cu_seqlens.cpu().numpy()
+    self_idx, self_kept = oracle.select(s, cu, spec.recent, B)
+    np.testing.assert_array_equal(gpu["idx"], self_idx)
+    np.testing.assert_array_equal(gpu["kept"], self_kept)
+    assert_compaction(lay, gpu, B)
