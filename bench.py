@@ -191,8 +191,9 @@ class ClockSampler:
         self.path = None
 
     def start(self):
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="waits_clocks_", suffix=".csv")
+        os.close(fd)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
@@ -203,6 +204,11 @@ class ClockSampler:
 
     def stop(self):
         if not self.proc:
+            if self.path:
+                try:
+                    os.remove(self.path)
+                except OSError:
+                    pass
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         try:
@@ -223,6 +229,10 @@ class ClockSampler:
             for name, v in zip(self.NAMES, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(name)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
                 "power_w_median": statistics.median(power) if power else None,
