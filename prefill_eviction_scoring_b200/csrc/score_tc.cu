@@ -516,6 +516,10 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
   const int t = tid & 127;                    // TMEM lane == row (pass 1) / key (pass 2)
   const int lane = tid & 31;
   const uint32_t lane_addr = tmem + ((uint32_t)((t >> 5) * 32) << 16);
+  // pass 1: this lane's packed row is token t / G of its Q tile (none past
+  // the tile's tokq * G rows); the division is done once here
+  const int t_tok = t / p.G;
+  const bool t_row = t < p.tokq * p.G;
   uint32_t kp = 0;          // pairs consumed by this warpgroup
   int sstep = 0;            // streamed steps seen (double-buffered shared data)
   bool ok = true;           // false after a timeout: keep every barrier, skip the work
@@ -525,6 +529,15 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
     const SeqInfo si = p.seqs[e.seq];
     const int g = e.g;
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};   // P1 row state / P2K sums
+    // pass 1: this lane's token in each of its stationary Q tiles (-1: no row)
+    int row_tok[2] = {-1, -1};
+    if (PASS == 1) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int tok = si.q0 + (e.stat0 + wg + 2 * k) * p.tokq + t_tok;
+        row_tok[k] = t_row && tok < si.len ? tok : -1;
+      }
+    }
     bar_sync(kBarAll, kEpiThreads);   // the previous unit's shared data is no longer read
     if (PASS == 2 && e.mode == kModeP2Q) {
       static_assert(kMaxStat == 2 * kWGs, "two stationary slots per warpgroup");
@@ -572,9 +585,8 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.tempty[buf]);
         if (PASS == 1) {
-          const int tok = si.q0 + j * p.tokq + t / p.G;
-          const bool row_ok = t < p.tokq * p.G && tok < si.len;
-          int nv = row_ok ? tok - kt * kTile + 1 : 0;
+          // in pass 1, j == e.stat0 + i: the token was found at the unit's start
+          int nv = row_tok[k] >= 0 ? row_tok[k] - kt * kTile + 1 : 0;
           nv = nv > kTile ? kTile : nv;
           p1_pair(v, nv, p.scale2, m[k], l[k]);
         } else {
