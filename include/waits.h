@@ -18,6 +18,9 @@
  *   Memory    Every pointer is DEVICE memory owned by the caller unless its
  *             comment says HOST.  The library allocates nothing and keeps no
  *             state between calls; scratch lives in the caller's workspace.
+ *             The one exception is waits_score_static (below): its scratch
+ *             is a fixed array inside the library, one per device, shared by
+ *             every call on that device, so those calls must be serialised.
  *             Q, K, V must be 16-byte aligned.
  *   Streams   `stream` is a cudaStream_t passed as void* (NULL = legacy
  *             default stream).  Calls only enqueue work on it and return; the
@@ -247,16 +250,28 @@ waits_status waits_compress_host(const waits_shape* shape,
  *   waits_workspace_size(shape) exceeds WAITS_STATIC_WORKSPACE_BYTES (nothing
  *   is launched).
  *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.
+ *   (cudaGetSymbolAddress, with that device current) and caches it for the
+ *   device's current CUDA context; a new context (after cudaDeviceReset, for
+ *   instance) looks it up again.  Make the first call on a device before any
+ *   stream capture.
  *   Every call on a device shares the one array, which keeps the previous
- *   call's contents; each call rewrites all of it before use.  Calls whose
- *   work overlaps on the GPU (other streams, other host threads) race on it:
- *   serialise them.  The device status word of this call lives in the array
- *   and is not readable through waits_read_device_status.
+ *   call's contents; every part of it a call reads is written earlier in
+ *   that call, so nothing needs clearing.  Calls whose work overlaps on the
+ *   GPU (other streams, other host threads) race on it: serialise them.
+ *   The call's device status word lives in the array: read it with
+ *   waits_read_static_status.
  */
 waits_status waits_score_static(const waits_shape* shape, const void* Q, const void* K,
                                 float a, int32_t b, float* scores, void* stream);
+
+/*
+ * Synchronise `stream` and read the device status word that the last
+ * waits_score_static call on the current device left in the library's
+ * static scratch (bits WAITS_DEV_*; 0 = clean).  Like that entry point, it
+ * has no counterpart on the WAITS pages.  Errors: ARG (status_bits NULL),
+ * CUDA.
+ */
+waits_status waits_read_static_status(void* stream, uint32_t* status_bits);
 
 /*
  * Synchronise `stream` and read the device status word of `workspace`
@@ -266,6 +281,26 @@ waits_status waits_score_static(const waits_shape* shape, const void* Q, const v
 waits_status waits_read_device_status(const void* workspace,
                                       size_t workspace_bytes, void* stream,
                                       uint32_t* status_bits);
+
+/*
+ * Testing aid, no counterpart on the WAITS pages: y[i] = the scorer's
+ * FMA-pipe 2^x of x[i] (the exponential that part of the scorer's epilogue
+ * runs instead of the MUFU ex2: a round-to-nearest split x = n + f, a cubic
+ * in f with relative error 1.013e-4 (1.02e-4 with fp32 rounding), 2^n
+ * added to the exponent; x is first clamped to [-125, 127]).  x and y are
+ * DEVICE fp32 arrays of n elements.  Errors: ARG (null pointer, n < 0),
+ * CUDA.
+ */
+waits_status waits_test_exp2_poly(const float* x, float* y, int64_t n, void* stream);
+
+/*
+ * Environment variables read at each waits_score / waits_compress call
+ * (testing aids): WAITS_WAIT_LIMIT_NS sets the limit of the scorer's
+ * bounded waits in nanoseconds (default 2 s); WAITS_TEST_WITHHOLD_MMA=1
+ * makes the scorer's MMA warp issue nothing, so the waits for its
+ * accumulators run out: the call ends early, with WAITS_DEV_TIMEOUT set and
+ * the scores unspecified, and leaves the context usable.
+ */
 
 #ifdef __cplusplus
 }

@@ -69,6 +69,8 @@ SIGNATURES = {
     "waits_read_device_status": (_I, [_P, _SZ, _P,
                                       ctypes.POINTER(ctypes.c_uint32)]),
     "waits_score_static": (_I, [_PSHAPE, _P, _P, _F, _I, _P, _P]),
+    "waits_read_static_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "waits_test_exp2_poly": (_I, [_P, _P, ctypes.c_int64, _P]),
     "waits_score_kernels": (_I, [_PSHAPE, _F, _I, ctypes.POINTER(ctypes.c_int32)]),
     "waits_select_compact": (_I, [_PSHAPE, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
 }

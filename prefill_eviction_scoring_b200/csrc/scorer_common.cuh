@@ -1,0 +1,386 @@
+// Pieces shared by the WAITS scorer kernels (score_tc.cu: every plan;
+// score_sparse.cu: the small plans of the sparse-weight regime): thread
+// roles and register split, the epilogue arithmetic (exponential sums over
+// a TMEM row of accumulators, the FMA-pipe 2^x), the merge of pass-1 row
+// partials into pass-2 row biases, the in-CTA work plan, and the TMA tensor
+// maps of the packed Q and K tensors.
+#pragma once
+
+#include "plan_core.cuh"
+#include "sm100.cuh"
+#include "unit_iter.cuh"
+
+namespace waits {
+namespace scorer {
+
+using namespace sm100;
+
+constexpr int kWGs = 2;                              // epilogue warpgroups
+constexpr int kEpiThreads = kWGs * 128;
+constexpr int kThreads = kEpiThreads + 128;          // + producer/MMA warpgroup
+// Register split (setmaxnreg): launched at 168 per thread (3 warps per SM
+// quadrant); the producer/MMA warpgroup drops to 56 and the two epilogue
+// warpgroups rise to 224: 128*56 + 256*224 = 384*168.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsProducer = 56;
+constexpr int kRegsEpilogue = 224;
+static_assert(128 * kRegsProducer + kEpiThreads * kRegsEpilogue <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
+constexpr int kProducerWarp = kWGs * 4;
+constexpr int kMmaWarp = kProducerWarp + 1;
+constexpr int kTmemCols = 512;
+constexpr uint64_t kDoneLimitNs = 2000000000ull;   // 2 s for the MMAs a CTA issued
+constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s after an abort
+constexpr int kBarAll = 3;                           // named barrier of both epilogue WGs
+
+__device__ inline float u2f(uint32_t v) { return __uint_as_float(v); }
+
+// ------------------------------------------------------------ epilogue ---
+// 128 accumulator columns of this thread's TMEM lane: the load and its wait
+// in one statement, so no use of the registers can be scheduled before the
+// data has arrived and the registers need no read-write operands (which can
+// cost a copy of each).
+struct Cols {
+  uint32_t r[128];
+  __device__ void load_wait(uint32_t taddr) {
+#define W8(b) "=r"(r[b]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), \
+              "=r"(r[b + 5]), "=r"(r[b + 6]), "=r"(r[b + 7])
+    asm volatile(
+        "{\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "}"
+        : W8(0), W8(8), W8(16), W8(24), W8(32), W8(40), W8(48), W8(56),
+          W8(64), W8(72), W8(80), W8(88), W8(96), W8(104), W8(112), W8(120)
+        : "r"(taddr)
+        : "memory");
+#undef W8
+  }
+};
+
+__device__ inline float2 f2(float x, float y) { return make_float2(x, y); }
+__device__ inline float hsum8(const float2 (&a)[4]) {
+  const float2 s = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+  return s.x + s.y;
+}
+
+// Column pairs whose exponential runs on the FMA pipe instead of the MUFU
+// (which does 16 ex2 per clock per SM and bounds the unmasked passes): bit
+// (pair index mod 8) of this mask.  One in eight measured best here (the
+// epilogue is latency-bound rather than MUFU-bound in this kernel; two in
+// eight was within 1.5%, three in eight 6% slower).
+constexpr uint32_t kPolyPairs = 0x80u;
+__device__ constexpr bool poly_col(int c) { return (kPolyPairs >> ((c >> 1) & 7)) & 1u; }
+
+// 2^x for a pair of fp32 values on the FMA/ALU pipes (Cody-Waite split plus
+// a polynomial): x = n + f with n = rint(x) and f in [-1/2, 1/2];
+// 2^f ~ 1 + f (c1 + f (c2 + f c3)), the relative-error minimax cubic with the
+// constant term held at 1 (max relative error 1.013e-4; fitted by linear
+// programming on a dense grid), so integer x gives exact powers of two; 2^n
+// is added to the exponent bits.  x is clamped to [-125, 127] so the result
+// stays a normal fp32 number.
+__device__ inline float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.0f;              // 1.5 * 2^23: rint via fadd
+  constexpr float c1 = 0.69328290f, c2 = 0.24221097f, c3 = 0.05500906f;
+  x = f2(fminf(fmaxf(x.x, -125.f), 127.f), fminf(fmaxf(x.y, -125.f), 127.f));
+  const float2 t = __fadd2_rn(x, f2(kMagic, kMagic));
+  const float2 n = __fadd2_rn(t, f2(-kMagic, -kMagic));
+  const float2 fr = __ffma2_rn(n, f2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(f2(c3, c3), fr, f2(c2, c2));
+  q = __ffma2_rn(q, fr, f2(c1, c1));
+  q = __ffma2_rn(q, fr, f2(1.f, 1.f));
+  // the magic's low 9 bits are zero, so (bits(t) << 23) == n << 23
+  const int ex = __float_as_int(t.x) << 23, ey = __float_as_int(t.y) << 23;
+  return f2(__int_as_float(__float_as_int(q.x) + ex), __int_as_float(__float_as_int(q.y) + ey));
+}
+
+// sum_c 2^(v_c * sc + off) over all 128 columns, packed fp32x2 arithmetic;
+// the column pairs picked by kPolyPairs use the polynomial, the rest the MUFU.
+__device__ inline float exp_sum_full(const Cols& v, float sc, float off) {
+  const float2 sc2 = f2(sc, sc), off2 = f2(off, off);
+  float2 a[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) a[k] = f2(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < kTile; c += 2) {
+    const float2 x = __ffma2_rn(f2(u2f(v.r[c]), u2f(v.r[c + 1])), sc2, off2);
+    const float2 e = poly_col(c) ? exp2_poly2(x) : f2(ex2_approx(x.x), ex2_approx(x.y));
+    a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], e);
+  }
+  return hsum8(a);
+}
+
+// Pass 1, one 128-key tile of this thread's row (keys c < nv are causal):
+// l += sum_c 2^(v_c*scale2 - m), m = first maximum seen, moved up only when
+// the running sum would leave the safe fp32 range.
+__device__ inline void p1_pair(const Cols& v, int nv, float sc, float& m, float& l) {
+  // one path per warp: a warp whose rows are not all fully causal (or absent)
+  // takes the masked path, which also serves its full rows
+  const bool full_warp = __all_sync(0xffffffffu, nv == kTile || nv <= 0);
+  if (nv <= 0) return;
+  if (m == -INFINITY) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, c < nv ? u2f(v.r[c]) * sc : -INFINITY);
+    m = mx;
+  }
+  float t;
+  if (full_warp) {
+    t = exp_sum_full(v, sc, -m);
+  } else {
+    const float nm = -m;
+    float a[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = 0.f;
+#pragma unroll
+    for (int c = 0; c < kTile; ++c) {
+      const float x = fmaf(u2f(v.r[c]), sc, nm);
+      a[c & 7] += ex2_approx(c < nv ? x : -INFINITY);
+    }
+    t = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+  }
+  if (l + t <= kRebaseLimit) {
+    l += t;
+    return;
+  }
+  // a value far above the reference: rebase on this tile's maximum
+  float mx = m;
+#pragma unroll
+  for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, c < nv ? u2f(v.r[c]) * sc : -INFINITY);
+  float t2 = 0.f;
+#pragma unroll
+  for (int c = 0; c < kTile; ++c) {
+    const float x = fmaf(u2f(v.r[c]), sc, -mx);
+    t2 += ex2_approx(c < nv ? x : -INFINITY);
+  }
+  l = l * ex2_approx(m - mx) + t2;
+  m = mx;
+}
+
+// Pass 2, one 128-row Q tile for this thread's key: sum over columns
+// c in [c_lo, ncols) of 2^(v_c*scale2 + bias_c) (bias is -inf past the rows).
+__device__ inline float p2_pair(const Cols& v, int c_lo, int ncols, float sc, const float* bias) {
+  const float4* b4 = reinterpret_cast<const float4*>(bias);
+  if (__all_sync(0xffffffffu, c_lo == 0)) {   // one path per warp
+    const float2 sc2 = f2(sc, sc);
+    float2 a[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) a[k] = f2(0.f, 0.f);
+#pragma unroll
+    for (int cb = 0; cb < kTile; cb += 32) {
+      if (cb < ncols) {
+#pragma unroll
+        for (int c = cb; c < cb + 32; c += 4) {
+          const float4 b = b4[c / 4];
+          const float2 x0 = __ffma2_rn(f2(u2f(v.r[c]), u2f(v.r[c + 1])), sc2, f2(b.x, b.y));
+          const float2 x1 = __ffma2_rn(f2(u2f(v.r[c + 2]), u2f(v.r[c + 3])), sc2, f2(b.z, b.w));
+          const float2 e0 = poly_col(c) ? exp2_poly2(x0) : f2(ex2_approx(x0.x), ex2_approx(x0.y));
+          const float2 e1 =
+              poly_col(c + 2) ? exp2_poly2(x1) : f2(ex2_approx(x1.x), ex2_approx(x1.y));
+          a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], e0);
+          a[((c >> 1) + 1) & 3] = __fadd2_rn(a[((c >> 1) + 1) & 3], e1);
+        }
+      }
+    }
+    return hsum8(a);
+  }
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = 0.f;
+#pragma unroll
+  for (int cb = 0; cb < kTile; cb += 32) {
+    if (cb < ncols) {
+#pragma unroll
+      for (int c = cb; c < cb + 32; c += 4) {
+        const float4 b = b4[c / 4];
+        const float x0 = fmaf(u2f(v.r[c + 0]), sc, b.x);
+        const float x1 = fmaf(u2f(v.r[c + 1]), sc, b.y);
+        const float x2 = fmaf(u2f(v.r[c + 2]), sc, b.z);
+        const float x3 = fmaf(u2f(v.r[c + 3]), sc, b.w);
+        a[(c + 0) & 7] += ex2_approx(c + 0 >= c_lo ? x0 : -INFINITY);
+        a[(c + 1) & 7] += ex2_approx(c + 1 >= c_lo ? x1 : -INFINITY);
+        a[(c + 2) & 7] += ex2_approx(c + 2 >= c_lo ? x2 : -INFINITY);
+        a[(c + 3) & 7] += ex2_approx(c + 3 >= c_lo ? x3 : -INFINITY);
+      }
+    }
+  }
+  return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+}
+
+__device__ inline void bar_sync(int id, int n) {
+  __syncwarp();
+  named_bar_sync(id, n);
+}
+// Named barrier that also ORs `v` over its threads (a uniform answer).
+__device__ inline bool bar_vote_or(int id, int n, bool v) {
+  __syncwarp();
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// Merge two (reference max, sum) pairs of the same row.
+__device__ inline float2 lse_merge(float2 x, float2 y) {
+  if (!(y.y > 0.f)) return x;
+  if (!(x.y > 0.f)) return y;
+  const float M = fmaxf(x.x, y.x);
+  return make_float2(M, x.y * ex2_approx(x.x - M) + y.y * ex2_approx(y.x - M));
+}
+
+// Bias of packed row r of the Q tiles j[k] (j[k] < 0: none; -inf where no
+// row exists): log2 of the row's curve weight minus its log2-sum-exp over
+// the keys, from the pass-1 partials of the row's units.  The partials of
+// all NR rows are loaded together (kMergeBatch units per row in flight) and
+// merged in unit order as a maximum, then a sum of the rescaled partial sums.
+template <int NR>
+__device__ inline void qrow_bias(const PassArgs& p, const SeqInfo& si, int g, const int (&j)[NR],
+                                 int r, float (&out)[NR]) {
+  constexpr size_t kStride = (size_t)kMaxStat1 * kTile;
+  constexpr int kMergeBatch = 16;
+  const int ngrp = (si.nqt + kMaxStat1 - 1) / kMaxStat1;     // pass-1 groups per head
+  const float2* src[NR];
+  int nu[NR], tok[NR], numax = 0;
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    tok[k] = si.q0 + j[k] * p.tokq + r / p.G;
+    nu[k] = 0;
+    src[k] = p.part1;
+    if (j[k] >= 0 && r < p.tokq * p.G && tok[k] < si.len) {
+      const Entry& e = p.e1[si.e1 + g * ngrp + j[k] / kMaxStat1];
+      src[k] = p.part1 + ((size_t)e.unit_base * kMaxStat1 + j[k] % kMaxStat1) * kTile + r;
+      nu[k] = e.n_units;
+    }
+    numax = max(numax, nu[k]);
+  }
+  float2 acc[NR];
+#pragma unroll
+  for (int k = 0; k < NR; ++k) acc[k] = make_float2(-INFINITY, 0.f);
+  for (int u0 = 0; u0 < numax; u0 += kMergeBatch) {
+    float2 x[NR][kMergeBatch];
+#pragma unroll
+    for (int k = 0; k < NR; ++k)
+#pragma unroll
+      for (int b = 0; b < kMergeBatch; ++b)
+        x[k][b] = u0 + b < nu[k] ? __ldcg(src[k] + (size_t)(u0 + b) * kStride)
+                                 : make_float2(-INFINITY, 0.f);
+#pragma unroll
+    for (int k = 0; k < NR; ++k) {
+      float M = acc[k].x;
+#pragma unroll
+      for (int b = 0; b < kMergeBatch; ++b)
+        if (x[k][b].y > 0.f) M = fmaxf(M, x[k][b].x);
+      float L = acc[k].y > 0.f ? acc[k].y * ex2_approx(acc[k].x - M) : 0.f;
+#pragma unroll
+      for (int b = 0; b < kMergeBatch; ++b)
+        if (x[k][b].y > 0.f) L += x[k][b].y * ex2_approx(x[k][b].x - M);
+      acc[k] = make_float2(M, L);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    const float w = nu[k] > 0 ? curve_weight(tok[k], si.len, p.a, p.b) : 0.f;
+    out[k] = w > 0.f ? log2f(w) - (acc[k].x + log2f(acc[k].y)) : -INFINITY;
+  }
+}
+
+// Every CTA's share of the plan: with a local plan each CTA builds it in
+// shared memory (or copies the host's one-sequence plan) and points `p` at
+// it; pass 1 also resets the call's status word and zeroes the scores of
+// sequences without an active row.  Called by all threads of the CTA.
+__device__ inline void plan_prologue(PassArgs& p, const PassArgs& pa, const HostPlan& hp,
+                                     LocalPlan* lp, bool p1, int warp) {
+  if (p.local_plan) {
+    // every CTA plans for itself (cu_seqlens is complete: pass 1 has waited
+    // above, and pass 2 starts only after pass 1 has), or copies the plan
+    // the host built for the batch {0, T} once cu_seqlens reads so
+    if (p.host_plan) {
+      const bool valid = p.cu[0] == 0 && p.cu[1] == p.T;   // the same two words in every thread
+      const int n1 = valid ? hp.hdr.n_e1 : 0, n2 = valid ? hp.hdr.n_e2 : 0;
+      constexpr int kVecs = (int)(sizeof(Entry) / sizeof(uint4));
+      const uint4* h1 = reinterpret_cast<const uint4*>(hp.e1);
+      const uint4* h2 = reinterpret_cast<const uint4*>(hp.e2);
+      uint4* d1 = reinterpret_cast<uint4*>(lp->e1);
+      uint4* d2 = reinterpret_cast<uint4*>(lp->e2);
+      for (int i = threadIdx.x; i < (n1 + n2) * kVecs; i += blockDim.x) {
+        if (i < n1 * kVecs) d1[i] = h1[i];
+        else d2[i - n1 * kVecs] = h2[i - n1 * kVecs];
+      }
+      if (threadIdx.x == 0) {
+        lp->seqs[0] = hp.seq;
+        PlanHeader h = hp.hdr;
+        if (!valid) {
+          h = PlanHeader{};
+          h.status = WAITS_DEV_BAD_SEQLENS;
+        }
+        lp->hdr = h;
+      }
+    } else if (warp == 0) {
+      warp_plan(p.cu, p.nseq, p.T, p.max_seqlen, p.Hkv, p.tokq, p.a, p.b, (int)gridDim.x, !p1,
+                *lp);
+    }
+    __syncthreads();
+    p.hdr = &lp->hdr;
+    p.seqs = lp->seqs;
+    p.e1 = lp->e1;
+    p.e2 = lp->e2;
+    if (p1) {
+      // this call's device status word, and zero scores for sequences
+      // without an active row (the planner kernel's duties)
+      if (blockIdx.x == 0 && threadIdx.x == 0) *pa.status = lp->hdr.status;
+      if (lp->hdr.status == 0) {
+        const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+        for (int q = 0; q < p.nseq; ++q) {
+          const SeqInfo si = lp->seqs[q];
+          if (si.len == 0 || si.q0 < si.len) continue;
+          for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+               i < (int64_t)si.len * p.Hkv; i += stride)
+            p.scores[(i / si.len) * p.T + si.start + i % si.len] = 0.0f;
+        }
+      }
+    }
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D view [T][heads][d] of a packed bf16 tensor; box = 64 x box_h x box_t.
+inline bool make_map(CUtensorMap* m, const void* base, int T, int heads, int d, int box_h, int box_t) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
+  const cuuint32_t box[3] = {64u, (cuuint32_t)box_h, (cuuint32_t)box_t};
+  const cuuint32_t elem[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+
+}  // namespace scorer
+}  // namespace waits

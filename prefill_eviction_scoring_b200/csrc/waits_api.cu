@@ -76,6 +76,23 @@ bool host_plan_allowed() {
   return !(force && force[0] == '1');
 }
 
+// WAITS_WAIT_LIMIT_NS (testing aid): limit of the scorer's bounded waits in
+// nanoseconds, default 2 s.  WAITS_TEST_WITHHOLD_MMA=1 (testing aid): the
+// scorer's MMA warp issues nothing, so the waits for its accumulators run out
+// and the call ends with WAITS_DEV_TIMEOUT set.
+uint64_t wait_limit_ns() {
+  const char* v = std::getenv("WAITS_WAIT_LIMIT_NS");
+  if (!v || !v[0]) return 2000000000ull;
+  char* end = nullptr;
+  const unsigned long long x = std::strtoull(v, &end, 10);
+  return end && *end == '\0' && x > 0 ? (uint64_t)x : 2000000000ull;
+}
+
+bool withhold_mma() {
+  const char* v = std::getenv("WAITS_TEST_WITHHOLD_MMA");
+  return v && v[0] == '1';
+}
+
 bool local_plan_fits(const waits_shape* s, float a, int32_t b) {
   // WAITS_PLANNER_KERNEL=1 (debugging, tests): always plan with the planner kernel
   const char* force = std::getenv("WAITS_PLANNER_KERNEL");
@@ -154,6 +171,8 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   p.scores = scores;
   p.status = &pa.hdr->status;
   p.local_plan = local ? 1 : 0;
+  p.wait_ns = wait_limit_ns();
+  p.withhold_mma = withhold_mma() ? 1 : 0;
   p.cu = s->cu_seqlens;
   p.nseq = s->nseq;
   p.max_seqlen = s->max_seqlen;
@@ -405,6 +424,14 @@ waits_status waits_compress_host(const waits_shape* shape, const int32_t* cu_hos
   if (!ok) return WAITS_ERR_CUDA;
   if (h2d_bytes) *h2d_bytes = up;
   if (d2h_bytes) *d2h_bytes = down;
+  return WAITS_OK;
+}
+
+waits_status waits_test_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  if (!x || !y || n < 0) return WAITS_ERR_ARG;
+  if (n == 0) return WAITS_OK;
+  const cudaError_t err = launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail("exp2 test launch", err);
   return WAITS_OK;
 }
 

@@ -242,6 +242,10 @@ struct PassArgs {
   int host_plan;
   const int32_t* cu;
   int nseq, max_seqlen;
+  // limit of every bounded wait in the main loops (ns); testing aid: with
+  // withhold_mma the MMA warp issues nothing, so those waits run out
+  uint64_t wait_ns;
+  int withhold_mma;
 };
 
 // ------------------------------------------- programmatic dependent launch ---
@@ -301,6 +305,7 @@ cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
 struct HostPlan;
 // hp: the host-built plan when a.host_plan (else unused, may be null).
 cudaError_t launch_score_passes(const PassArgs& a, const HostPlan* hp, int grid, cudaStream_t s);
+cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
 // K == nullptr: selection only; else also the compaction of K and V into
 // Ko, Vo (the rows of the kept positions, zeros past kept_len).
 cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int T,

@@ -72,3 +72,30 @@ def test_full_size_layer_fits_the_static_scratch():
     out = api.score_static(lay.Q, lay.K, lay.cu_seqlens, sigmoid_a=1.0, window=16)
     torch.cuda.synchronize()
     assert_scores_close(out.double().cpu().numpy(), ref.double().cpu().numpy())
+
+
+@pytest.mark.gpu
+def test_static_status_word_reports_bad_seqlens_then_clears():
+    """A malformed cu_seqlens handed to waits_score_static sets the bad-offsets
+    bit of the status word in the library's static scratch, which
+    waits_read_static_status reads; the next well-formed call clears it."""
+    lib = _lib.load()
+    lay = wl.make_layer("tiny", lens=(300,), device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    out = torch.empty((lay.K.shape[1], lay.total_tokens), device="cuda")
+    st = ctypes.c_uint32(0)
+    bad_cu = torch.tensor([0, lay.total_tokens - 7], dtype=torch.int32, device="cuda")
+    T, Hq, d = lay.Q.shape
+    bad = api.make_shape(bad_cu, T, lay.max_seqlen, Hq, lay.K.shape[1], d)
+    _lib.check("waits_score_static", lib.waits_score_static(
+        ctypes.byref(bad), lay.Q.data_ptr(), lay.K.data_ptr(), 1.0, 16, out.data_ptr(), stream))
+    _lib.check("waits_read_static_status", lib.waits_read_static_status(stream, ctypes.byref(st)))
+    assert st.value & _lib.DEV_BAD_SEQLENS
+    _lib.check("waits_score_static", _score_static_raw(lib, lay, 1.0, 16, out))
+    _lib.check("waits_read_static_status", lib.waits_read_static_status(stream, ctypes.byref(st)))
+    assert st.value == 0
+
+
+def test_static_status_reader_rejects_null():
+    lib = _lib.load()
+    assert lib.waits_read_static_status(None, None) == 1
