@@ -299,7 +299,9 @@ waits_status waits_test_exp2_poly(const float* x, float* y, int64_t n, void* str
  * bounded waits in nanoseconds (default 2 s); WAITS_TEST_WITHHOLD_MMA=1
  * makes the scorer's MMA warp issue nothing, so the waits for its
  * accumulators run out: the call ends early, with WAITS_DEV_TIMEOUT set and
- * the scores unspecified, and leaves the context usable.
+ * the scores unspecified, and leaves the context usable.  WAITS_SCORER=tc
+ * makes small plans run the general scorer kernel instead of the one for
+ * sparse weights (the scores are bit-identical either way).
  */
 
 #ifdef __cplusplus

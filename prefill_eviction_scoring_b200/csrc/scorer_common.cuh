@@ -19,11 +19,12 @@ constexpr int kWGs = 2;                              // epilogue warpgroups
 constexpr int kEpiThreads = kWGs * 128;
 constexpr int kThreads = kEpiThreads + 128;          // + producer/MMA warpgroup
 // Register split (setmaxnreg): launched at 168 per thread (3 warps per SM
-// quadrant); the producer/MMA warpgroup drops to 56 and the two epilogue
-// warpgroups rise to 224: 128*56 + 256*224 = 384*168.
+// quadrant); the producer/MMA warpgroup drops to 104 and the two epilogue
+// warpgroups rise to 200: 128*104 + 256*200 = 384*168 - 2048.  (56 for the
+// copy and MMA warps made them spill in their loops; measured 1 % slower.)
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsProducer = 56;
-constexpr int kRegsEpilogue = 224;
+constexpr int kRegsProducer = 104;
+constexpr int kRegsEpilogue = 200;
 static_assert(128 * kRegsProducer + kEpiThreads * kRegsEpilogue <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr int kProducerWarp = kWGs * 4;
@@ -240,8 +241,8 @@ __device__ inline float2 lse_merge(float2 x, float2 y) {
 // all NR rows are loaded together (kMergeBatch units per row in flight) and
 // merged in unit order as a maximum, then a sum of the rescaled partial sums.
 template <int NR>
-__device__ inline void qrow_bias(const PassArgs& p, const SeqInfo& si, int g, const int (&j)[NR],
-                                 int r, float (&out)[NR]) {
+__device__ inline void qrow_bias(const PassArgs& p, const Entry* e1, const SeqInfo& si, int g,
+                                 const int (&j)[NR], int r, float (&out)[NR]) {
   constexpr size_t kStride = (size_t)kMaxStat1 * kTile;
   constexpr int kMergeBatch = 16;
   const int ngrp = (si.nqt + kMaxStat1 - 1) / kMaxStat1;     // pass-1 groups per head
@@ -253,7 +254,7 @@ __device__ inline void qrow_bias(const PassArgs& p, const SeqInfo& si, int g, co
     nu[k] = 0;
     src[k] = p.part1;
     if (j[k] >= 0 && r < p.tokq * p.G && tok[k] < si.len) {
-      const Entry& e = p.e1[si.e1 + g * ngrp + j[k] / kMaxStat1];
+      const Entry& e = e1[si.e1 + g * ngrp + j[k] / kMaxStat1];
       src[k] = p.part1 + ((size_t)e.unit_base * kMaxStat1 + j[k] % kMaxStat1) * kTile + r;
       nu[k] = e.n_units;
     }
@@ -288,6 +289,13 @@ __device__ inline void qrow_bias(const PassArgs& p, const SeqInfo& si, int g, co
     const float w = nu[k] > 0 ? curve_weight(tok[k], si.len, p.a, p.b) : 0.f;
     out[k] = w > 0.f ? log2f(w) - (acc[k].x + log2f(acc[k].y)) : -INFINITY;
   }
+}
+
+// The same, with the pass-1 entries of the plan `p` points at.
+template <int NR>
+__device__ inline void qrow_bias(const PassArgs& p, const SeqInfo& si, int g, const int (&j)[NR],
+                                 int r, float (&out)[NR]) {
+  qrow_bias<NR>(p, p.e1, si, g, j, r, out);
 }
 
 // Every CTA's share of the plan: with a local plan each CTA builds it in

@@ -88,6 +88,13 @@ uint64_t wait_limit_ns() {
   return end && *end == '\0' && x > 0 ? (uint64_t)x : 2000000000ull;
 }
 
+// WAITS_SCORER=tc (debugging, tests): local plans also run the general
+// scorer kernel (128-column accumulators) instead of the sparse one.
+bool force_tc_scorer() {
+  const char* v = std::getenv("WAITS_SCORER");
+  return v && v[0] == 't' && v[1] == 'c' && v[2] == '\0';
+}
+
 bool withhold_mma() {
   const char* v = std::getenv("WAITS_TEST_WITHHOLD_MMA");
   return v && v[0] == '1';
@@ -181,7 +188,10 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
                         host_plan_single(p.T, p.max_seqlen, p.Hkv, p.tokq, a, b, grid, &hp)
                     ? 1
                     : 0;
-  err = launch_score_passes(p, p.host_plan ? &hp : nullptr, grid, st);
+  // local plans hold only P2Q entries in pass 2: the 256-column kernel
+  err = local && !force_tc_scorer()
+            ? launch_sparse_passes(p, p.host_plan ? &hp : nullptr, grid, st)
+            : launch_score_passes(p, p.host_plan ? &hp : nullptr, grid, st);
   if (err != cudaSuccess) return cuda_fail("scorer launch", err);
   return WAITS_OK;
 }

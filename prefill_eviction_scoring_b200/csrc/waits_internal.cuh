@@ -305,6 +305,9 @@ cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
 struct HostPlan;
 // hp: the host-built plan when a.host_plan (else unused, may be null).
 cudaError_t launch_score_passes(const PassArgs& a, const HostPlan* hp, int grid, cudaStream_t s);
+// The same two passes for a local plan (every entry of pass 2 in mode P2Q):
+// 256-column accumulators, bit-identical scores.
+cudaError_t launch_sparse_passes(const PassArgs& a, const HostPlan* hp, int grid, cudaStream_t s);
 cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
 // K == nullptr: selection only; else also the compaction of K and V into
 // Ko, Vo (the rows of the kept positions, zeros past kept_len).
