@@ -67,10 +67,9 @@ __device__ inline float hsum8(const float2 (&a)[4]) {
 
 // Column pairs whose exponential runs on the FMA pipe instead of the MUFU
 // (which does 16 ex2 per clock per SM and bounds the unmasked passes): bit
-// (pair index mod 8) of this mask.  One in eight measured best here (the
-// epilogue is latency-bound rather than MUFU-bound in this kernel; two in
-// eight was within 1.5%, three in eight 6% slower).
-constexpr uint32_t kPolyPairs = 0x80u;
+// (pair index mod 8) of this mask.  Two in eight measured best with the
+// 256-column accumulators (one in eight 3 % slower, three in eight 4 %).
+constexpr uint32_t kPolyPairs = 0x88u;
 __device__ constexpr bool poly_col(int c) { return (kPolyPairs >> ((c >> 1) & 7)) & 1u; }
 
 // 2^x for a pair of fp32 values on the FMA/ALU pipes (Cody-Waite split plus
