@@ -63,6 +63,7 @@ typedef enum waits_status {
 #define WAITS_DEV_BAD_SEQLENS    0x2u  /* cu_seqlens not 0 <= ... <= T, or N > max_seqlen */
 #define WAITS_DEV_PLAN_OVERFLOW  0x4u  /* internal: plan larger than its bound */
 #define WAITS_DEV_BAD_INDEX      0x8u  /* waits_compact saw idx outside [0, N) */
+#define WAITS_DEV_BAD_CURVE      0x10u /* a routed call's a or b was invalid for some sequence */
 
 typedef struct waits_shape {
   int32_t nseq;             /* sequences in the packed batch, >= 1             */
@@ -129,6 +130,51 @@ waits_status waits_score_kernels(const waits_shape* shape, float a, int32_t b,
 waits_status waits_score(const waits_shape* shape, const void* Q, const void* K,
                          float a, int32_t b, float* scores, void* workspace,
                          size_t workspace_bytes, void* stream);
+
+/*
+ * waits_score with the softmax normalisers supplied by the caller: the
+ * prefill attention that precedes the scorer (the README's opening summary
+ * has WAITS registered as an attention function, so it runs right after
+ * the layer's attention) has already computed every row's log-sum-exp, as a
+ * FlashAttention forward returns it.  The first pass (row statistics) is
+ * then skipped and only the weighted column sums run, half the work.
+ *   lse   DEVICE fp32 [Hq, T]: lse[h * T + t] = natural log of
+ *         sum_{k <= q} exp(Q[t,h] . K[k,g] / sqrt(d)), q the sequence-local
+ *         position of packed token t (keys of its own sequence only); read
+ *         only for rows whose fp32 weight is non-zero
+ *   other arguments, layouts and results as waits_score; with the exact
+ *   LSE the scores equal waits_score's within fp32 rounding.
+ * Errors: as waits_score, plus ARG if lse is NULL or not 4-byte aligned.
+ */
+waits_status waits_score_with_lse(const waits_shape* shape, const void* Q, const void* K,
+                                  const float* lse, float a, int32_t b, float* scores,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * waits_score with a forgetting curve per sequence: the README's routed
+ * WAITS ("Training the routing policy" and Evaluation's --waits_table) picks
+ * one (a, b) action per sample, so one packed batch mixes curves.
+ *   a     DEVICE fp32 [nseq]: slope of sequence i, finite and >= 0
+ *   b     DEVICE int32 [nseq]: window of sequence i, >= 0
+ *   other arguments, layouts and results as waits_score, each sequence
+ *   scored with its own (a[i], b[i]).  The work plan is built on the device
+ *   (3 kernels).  A sequence whose a or b is invalid sets WAITS_DEV_BAD_CURVE
+ *   and gets zero scores.
+ * Errors: as waits_score, plus ARG if a or b is NULL or misaligned.
+ */
+waits_status waits_score_routed(const waits_shape* shape, const void* Q, const void* K,
+                                const float* a, const int32_t* b, float* scores,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * waits_score_routed followed by waits_select_compact (per-sequence curves,
+ * then selection and compaction), all enqueued on `stream`.
+ */
+waits_status waits_compress_routed(const waits_shape* shape, const void* Q, const void* K,
+                                   const void* V, const float* a, const int32_t* b, int32_t R,
+                                   int32_t B, float* scores, int32_t* idx, int32_t* kept_len,
+                                   void* K_out, void* V_out, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /*
  * Selection (README Quickstart budgets).  Per sequence i and KV head g:

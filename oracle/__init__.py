@@ -18,6 +18,7 @@ sort, explicit loops). No function here is "parity unpinned".
 
 from .waits_oracle import (  # noqa: F401
     forgetting_curve,
+    row_lse,
     score,
     select,
     compact,

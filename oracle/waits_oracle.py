@@ -55,7 +55,7 @@ def _seq_bounds(cu_seqlens):
     return [(int(cu[i]), int(cu[i + 1])) for i in range(len(cu) - 1)]
 
 
-def score(Q, K, cu_seqlens, a, b, *, row_block=512):
+def score(Q, K, cu_seqlens, a, b, *, row_block=512, last=None):
     """Accumulative forgetting-curve attention score, fp64.
 
     For every sequence, query head h and KV head g = h // G:
@@ -65,6 +65,11 @@ def score(Q, K, cu_seqlens, a, b, *, row_block=512):
     Rows whose fp64 weight is exactly 0.0 are skipped; that is exact.
     Rows are processed in blocks of ``row_block`` only to bound memory: every
     row is an independent softmax, so the block size cannot change a value.
+
+    With ``last`` only the last ``last`` rows of each sequence are summed:
+    a key k receives attention only from rows q >= k, so the scores of the
+    last ``last`` keys of each sequence are then exact (the rest are partial
+    sums).  That makes long sequences checkable key by key at their tail.
 
     Returns ``s`` of shape ``[Hkv, T]`` (fp64), indexed by packed token.
     """
@@ -83,6 +88,8 @@ def score(Q, K, cu_seqlens, a, b, *, row_block=512):
             continue
         w = forgetting_curve(np.arange(N), N, a, b)
         rows = np.nonzero(w != 0.0)[0]
+        if last is not None:
+            rows = rows[rows >= N - int(last)]
         keys = np.arange(N)
         for h in range(Hq):
             g = h // G
@@ -96,6 +103,46 @@ def score(Q, K, cu_seqlens, a, b, *, row_block=512):
                 P = E / E.sum(axis=1, keepdims=True)
                 s[g, lo:hi] += (w[q][:, None] * P).sum(axis=0)
     return s
+
+
+def row_lse(Q, K, cu_seqlens, last=None):
+    """Natural-log log-sum-exp of every causal attention row, fp64.
+
+    ``lse[h, t] = log sum_{k <= q} exp(Q[t, h] . K[lo + k, g] / sqrt(d))``
+    for packed token ``t = lo + q`` of a sequence starting at ``lo``, with
+    g = h // G: the normaliser of the causal softmax whose probabilities the
+    WAITS score accumulates (opening summary).  It is what a FlashAttention
+    forward returns as its row LSE, and what the caller hands to the scorer
+    to skip the row-statistics pass.  Every row is computed, whatever its
+    weight, unless ``last`` is given: then only the last ``last`` rows of
+    each sequence are, and the others are NaN.
+
+    Returns ``lse`` of shape ``[Hq, T]`` (fp64).
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    T, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    if Hq % Hkv:
+        raise ValueError("query heads must be a multiple of KV heads")
+    G = Hq // Hkv
+    inv_sqrt_d = 1.0 / np.sqrt(float(d))
+    lse = np.full((Hq, T), np.nan if last is not None else 0.0, dtype=np.float64)
+    for lo, hi in _seq_bounds(cu_seqlens):
+        N = hi - lo
+        if N == 0:
+            continue
+        keys = np.arange(N)
+        first = 0 if last is None else max(0, N - int(last))
+        for h in range(Hq):
+            Kg = K[lo:hi, h // G, :]
+            for start in range(first, N, 512):
+                q = np.arange(start, min(N, start + 512))
+                L = (Q[lo + q, h, :] @ Kg.T) * inv_sqrt_d
+                L[keys[None, :] > q[:, None]] = -np.inf
+                m = L.max(axis=1)
+                lse[h, lo + q] = m + np.log(np.exp(L - m[:, None]).sum(axis=1))
+    return lse
 
 
 def select(s, cu_seqlens, R, B):

@@ -17,7 +17,7 @@ STATUS_NAMES = {0: "WAITS_OK", 1: "WAITS_ERR_ARG", 2: "WAITS_ERR_SHAPE",
                 3: "WAITS_ERR_UNSUPPORTED", 4: "WAITS_ERR_WORKSPACE",
                 5: "WAITS_ERR_CUDA", 6: "WAITS_ERR_TIMEOUT",
                 7: "WAITS_ERR_DEVICE"}
-DEV_TIMEOUT, DEV_BAD_SEQLENS, DEV_PLAN_OVERFLOW, DEV_BAD_INDEX = 1, 2, 4, 8
+DEV_TIMEOUT, DEV_BAD_SEQLENS, DEV_PLAN_OVERFLOW, DEV_BAD_INDEX, DEV_BAD_CURVE = 1, 2, 4, 8, 16
 
 
 class WaitsLibraryError(RuntimeError):
@@ -58,6 +58,10 @@ SIGNATURES = {
     "waits_last_error": (ctypes.c_char_p, []),
     "waits_workspace_size": (_I, [_PSHAPE, ctypes.POINTER(_SZ)]),
     "waits_score": (_I, [_PSHAPE, _P, _P, _F, _I, _P, _P, _SZ, _P]),
+    "waits_score_with_lse": (_I, [_PSHAPE, _P, _P, _P, _F, _I, _P, _P, _SZ, _P]),
+    "waits_score_routed": (_I, [_PSHAPE, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "waits_compress_routed": (_I, [_PSHAPE, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P,
+                                   _P, _SZ, _P]),
     "waits_select": (_I, [_PSHAPE, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "waits_compact": (_I, [_PSHAPE, _P, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "waits_compress": (_I, [_PSHAPE, _P, _P, _P, _F, _I, _I, _I, _P, _P, _P,

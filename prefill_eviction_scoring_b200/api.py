@@ -111,6 +111,50 @@ class Compressor:
         _lib.check("waits_score", st)
         return self.scores
 
+    def compress_routed(self, Q, K, V, sigmoid_a: torch.Tensor, window: torch.Tensor,
+                        recent_budget: int):
+        """``waits_compress_routed``: per-sequence curves, ``sigmoid_a`` fp32
+        ``[nseq]`` and ``window`` int32 ``[nseq]`` on the device."""
+        self.check_inputs(Q, K, V)
+        _need_cuda("sigmoid_a", sigmoid_a, torch.float32)
+        _need_cuda("window", window, torch.int32)
+        if sigmoid_a.numel() != self.nseq or window.numel() != self.nseq:
+            raise ValueError("one sigmoid_a and one window per sequence")
+        st = self.lib.waits_compress_routed(
+            ctypes.byref(self.shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(sigmoid_a), _ptr(window),
+            int(recent_budget), self.B, _ptr(self.scores), _ptr(self.idx), _ptr(self.kept_len),
+            _ptr(self.K_out), _ptr(self.V_out), _ptr(self.workspace), self.ws_bytes,
+            _stream(self.dev))
+        _lib.check("waits_compress_routed", st)
+        return self.K_out, self.V_out, self.idx, self.kept_len, self.scores
+
+    def score_routed(self, Q, K, sigmoid_a: torch.Tensor, window: torch.Tensor):
+        """``waits_score_routed``: per-sequence ``sigmoid_a`` (fp32) and
+        ``window`` (int32) device tensors of ``nseq`` values."""
+        self.check_inputs(Q, K)
+        _need_cuda("sigmoid_a", sigmoid_a, torch.float32)
+        _need_cuda("window", window, torch.int32)
+        if sigmoid_a.numel() != self.nseq or window.numel() != self.nseq:
+            raise ValueError("one sigmoid_a and one window per sequence")
+        st = self.lib.waits_score_routed(
+            ctypes.byref(self.shape), _ptr(Q), _ptr(K), _ptr(sigmoid_a), _ptr(window),
+            _ptr(self.scores), _ptr(self.workspace), self.ws_bytes, _stream(self.dev))
+        _lib.check("waits_score_routed", st)
+        return self.scores
+
+    def score_with_lse(self, Q, K, lse, sigmoid_a: float, window: int):
+        """``waits_score_with_lse``: the scores from the caller's row LSE
+        (fp32 ``[Hq, T]``, natural log), without the row-statistics pass."""
+        self.check_inputs(Q, K)
+        _need_cuda("lse", lse, torch.float32)
+        if tuple(lse.shape) != (self.Hq, self.T) or not lse.is_contiguous():
+            raise ValueError("lse must be a contiguous fp32 [Hq, T] tensor")
+        st = self.lib.waits_score_with_lse(
+            ctypes.byref(self.shape), _ptr(Q), _ptr(K), _ptr(lse), float(sigmoid_a), int(window),
+            _ptr(self.scores), _ptr(self.workspace), self.ws_bytes, _stream(self.dev))
+        _lib.check("waits_score_with_lse", st)
+        return self.scores
+
     def device_status(self) -> int:
         v = ctypes.c_uint32(0)
         _lib.check("waits_read_device_status", self.lib.waits_read_device_status(
@@ -124,6 +168,18 @@ def score(Q: torch.Tensor, K: torch.Tensor, cu_seqlens: torch.Tensor, *,
     T, Hq, d = Q.shape
     c = Compressor(cu_seqlens, T, _max_seqlen(cu_seqlens, max_seqlen), Hq, K.shape[1], d, 1)
     return c.score(Q, K, sigmoid_a, window)
+
+
+def score_with_lse(Q: torch.Tensor, K: torch.Tensor, cu_seqlens: torch.Tensor,
+                   lse: torch.Tensor, *, sigmoid_a: float, window: int,
+                   max_seqlen: Optional[int] = None) -> torch.Tensor:
+    """fp32 ``[Hkv, T]`` scores (``waits_score_with_lse``) from the caller's
+    natural-log row LSE ``[Hq, T]`` (a FlashAttention forward's
+    ``softmax_lse``): only the weighted column-sum pass runs."""
+    _need_cuda("cu_seqlens", cu_seqlens, torch.int32)
+    T, Hq, d = Q.shape
+    c = Compressor(cu_seqlens, T, _max_seqlen(cu_seqlens, max_seqlen), Hq, K.shape[1], d, 1)
+    return c.score_with_lse(Q, K, lse, sigmoid_a, window)
 
 
 def score_static(Q: torch.Tensor, K: torch.Tensor, cu_seqlens: torch.Tensor, *,

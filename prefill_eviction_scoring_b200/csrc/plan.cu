@@ -111,10 +111,10 @@ __device__ void plan_pass(const Seqs& S, int nseq, int tokq, int n, int grid, En
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs p) {
   __shared__ int64_t sh[32];
-  __shared__ int s_bad;
+  __shared__ int s_bad, s_bad_curve;
   __shared__ SeqInfo s_seqs[kSmemSeqs];
   const int tid = threadIdx.x;
-  if (tid == 0) s_bad = 0;
+  if (tid == 0) s_bad = s_bad_curve = 0;
   pdl_allow_next();
   pdl_wait();
   __syncthreads();
@@ -128,8 +128,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs p) {
     int64_t v1 = 0, v2 = 0;
     if (s < p.nseq) {
       bool bad;
-      si = seq_info(p.cu, s, p.nseq, p.T, p.max_seqlen, p.tokq, p.a, p.b, bad);
+      const float a = p.seq_a ? p.seq_a[s] : p.a;
+      const int b = p.seq_b ? p.seq_b[s] : p.b;
+      si = seq_info(p.cu, s, p.nseq, p.T, p.max_seqlen, p.tokq, a, b, bad);
       if (bad) atomicOr(&s_bad, 1);
+      if (!(a >= 0.0f && a <= 3.4e38f && b >= 0)) atomicOr(&s_bad_curve, 1);
       v1 = (int64_t)p.Hkv * groups_p1(si);
       v2 = (int64_t)p.Hkv * groups_p2(si);
     }
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs p) {
                      &P2, &A2, &overflow);
   }
   if (tid == 0) {
-    H->status = overflow ? WAITS_DEV_PLAN_OVERFLOW : 0u;
+    H->status = (overflow ? WAITS_DEV_PLAN_OVERFLOW : 0u) | (s_bad_curve ? WAITS_DEV_BAD_CURVE : 0u);
     H->n_e1 = overflow ? 0 : (int)c1;
     H->n_e2 = overflow ? 0 : (int)c2;
     H->n_u1 = U1;

@@ -35,9 +35,14 @@ __host__ __device__ inline SeqInfo seq_info(int lo, int hi, int s, int nseq, int
   SeqInfo si{};
   bad = (s == 0 && lo != 0) || hi < lo || hi > T || (hi - lo) > max_seqlen ||
         (s == nseq - 1 && hi != T);
+  // an invalid curve (only routed calls can pass one) leaves the sequence
+  // without active rows: its scores are zero
+  const bool curve_ok = a >= 0.0f && a <= 3.4e38f && b >= 0;
   si.start = lo;
   si.len = bad ? 0 : hi - lo;
-  si.q0 = first_active_row(si.len, a, b);
+  si.a = curve_ok ? a : 0.0f;
+  si.b = curve_ok ? b : 0;
+  si.q0 = curve_ok ? first_active_row(si.len, a, b) : si.len;
   si.nqt = (si.len - si.q0 + tokq - 1) / tokq;
   si.nkt = (si.len + kTile - 1) / kTile;
   return si;

@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Pass 1 waits for whatever wrote Q, K and cu_seqlens before anything,
   // then lets pass 2 launch; pass 2's copy and MMA warps start at once, only
   // its epilogue waits (below) for pass 1's row partials.
-  if (p1) {
+  if (p1 || pa.lse) {
     pdl_wait();
     pdl_allow_next();
   }
@@ -504,8 +504,8 @@ cudaError_t launch_sparse_d(const PassArgs& a, const HostPlan& hp, int grid, cud
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) !=
           cudaSuccess)
     return err;
-  if ((err = launch_pdl(score_sparse_kernel<D, 1>, dim3(grid), dim3(kThreads), smem1, st, mq, mk,
-                        a, hp)) != cudaSuccess)
+  if (!a.lse && (err = launch_pdl(score_sparse_kernel<D, 1>, dim3(grid), dim3(kThreads), smem1,
+                                  st, mq, mk, a, hp)) != cudaSuccess)
     return err;
   return launch_pdl(score_sparse_kernel<D, 2>, dim3(grid), dim3(kThreads), smem2, st, mq, mk, a,
                     hp);

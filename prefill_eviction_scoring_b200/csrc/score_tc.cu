@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // then lets pass 2 launch: from then on the plan, Q and K are complete, so
   // pass 2's copy and MMA warps start on them at once; only its epilogue
   // waits (below) for pass 1's row biases.
-  if (p1) {
+  if (p1 || pa.lse) {
     pdl_wait();
     pdl_allow_next();
   }
@@ -498,8 +498,8 @@ cudaError_t launch_d(const PassArgs& a, const HostPlan& hp, int grid, cudaStream
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) !=
           cudaSuccess)
     return err;
-  if ((err = launch_pdl(score_tc_kernel<D, 1>, dim3(grid), dim3(kThreads), smem1, st, mq, mk,
-                        a, hp)) != cudaSuccess) {
+  if (!a.lse && (err = launch_pdl(score_tc_kernel<D, 1>, dim3(grid), dim3(kThreads), smem1, st,
+                                  mq, mk, a, hp)) != cudaSuccess) {
     cudaFuncAttributes fa{};
     cudaFuncGetAttributes(&fa, score_tc_kernel<D, 1>);
     int dev = 0, optin = 0, regs = 0;

@@ -110,51 +110,60 @@ __device__ inline float exp_sum_full(const Cols& v, float sc, float off) {
   return hsum8(a);
 }
 
+// Largest of the tile's first nv values, scaled.
+__device__ inline float tile_max(const Cols& v, int nv, float sc) {
+  float mx = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, c < nv ? u2f(v.r[c]) * sc : -INFINITY);
+  return mx;
+}
+
+// sum over c < nv of 2^(v_c*sc + off) (masked tiles, MUFU only: exact zeros)
+__device__ inline float exp_sum_masked(const Cols& v, int nv, float sc, float off) {
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = 0.f;
+#pragma unroll
+  for (int c = 0; c < kTile; ++c) {
+    const float x = fmaf(u2f(v.r[c]), sc, off);
+    a[c & 7] += ex2_approx(c < nv ? x : -INFINITY);
+  }
+  return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+}
+
+// Largest raw value of the whole tile (8 independent chains).
+__device__ inline float tile_max_raw(const Cols& v) {
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = u2f(v.r[k]);
+#pragma unroll
+  for (int c = 8; c < kTile; ++c) mx[c & 7] = fmaxf(mx[c & 7], u2f(v.r[c]));
+  return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+}
+
 // Pass 1, one 128-key tile of this thread's row (keys c < nv are causal):
-// l += sum_c 2^(v_c*scale2 - m), m = first maximum seen, moved up only when
-// the running sum would leave the safe fp32 range.
+// l += sum_c 2^(v_c*scale2 - m) after moving the reference m up to the
+// tile's maximum when that is higher (rescaling l), so no term exceeds 1 and
+// the sum cannot overflow.  A masked tile takes the maximum of its causal
+// values only.
 __device__ inline void p1_pair(const Cols& v, int nv, float sc, float& m, float& l) {
   // one path per warp: a warp whose rows are not all fully causal (or absent)
   // takes the masked path, which also serves its full rows
   const bool full_warp = __all_sync(0xffffffffu, nv == kTile || nv <= 0);
   if (nv <= 0) return;
-  if (m == -INFINITY) {
-    float mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, c < nv ? u2f(v.r[c]) * sc : -INFINITY);
+  const float mx = full_warp ? tile_max_raw(v) * sc : tile_max(v, nv, sc);
+  if (mx > m) {
+    if (l > 0.f) l *= ex2_approx(m - mx);
     m = mx;
   }
   float t;
   if (full_warp) {
     t = exp_sum_full(v, sc, -m);
   } else {
-    const float nm = -m;
-    float a[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] = 0.f;
-#pragma unroll
-    for (int c = 0; c < kTile; ++c) {
-      const float x = fmaf(u2f(v.r[c]), sc, nm);
-      a[c & 7] += ex2_approx(c < nv ? x : -INFINITY);
-    }
-    t = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+    t = exp_sum_masked(v, nv, sc, -m);
   }
-  if (l + t <= kRebaseLimit) {
-    l += t;
-    return;
-  }
-  // a value far above the reference: rebase on this tile's maximum
-  float mx = m;
-#pragma unroll
-  for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, c < nv ? u2f(v.r[c]) * sc : -INFINITY);
-  float t2 = 0.f;
-#pragma unroll
-  for (int c = 0; c < kTile; ++c) {
-    const float x = fmaf(u2f(v.r[c]), sc, -mx);
-    t2 += ex2_approx(c < nv ? x : -INFINITY);
-  }
-  l = l * ex2_approx(m - mx) + t2;
-  m = mx;
+  l += t;
 }
 
 // Pass 2, one 128-row Q tile for this thread's key: sum over columns
@@ -242,6 +251,19 @@ __device__ inline float2 lse_merge(float2 x, float2 y) {
 template <int NR>
 __device__ inline void qrow_bias(const PassArgs& p, const Entry* e1, const SeqInfo& si, int g,
                                  const int (&j)[NR], int r, float (&out)[NR]) {
+  if (p.lse) {
+    // the caller's natural-log row LSE replaces pass 1: log2 w - lse * log2(e)
+    constexpr float kLog2e = 1.4426950408889634f;
+#pragma unroll
+    for (int k = 0; k < NR; ++k) {
+      const int tok = si.q0 + j[k] * p.tokq + r / p.G;
+      const bool row = j[k] >= 0 && r < p.tokq * p.G && tok < si.len;
+      const float w = row ? curve_weight(tok, si.len, si.a, si.b) : 0.f;
+      const size_t h = (size_t)g * p.G + r % p.G;
+      out[k] = w > 0.f ? log2f(w) - p.lse[h * p.T + si.start + tok] * kLog2e : -INFINITY;
+    }
+    return;
+  }
   constexpr size_t kStride = (size_t)kMaxStat1 * kTile;
   constexpr int kMergeBatch = 16;
   const int ngrp = (si.nqt + kMaxStat1 - 1) / kMaxStat1;     // pass-1 groups per head
@@ -285,7 +307,7 @@ __device__ inline void qrow_bias(const PassArgs& p, const Entry* e1, const SeqIn
   }
 #pragma unroll
   for (int k = 0; k < NR; ++k) {
-    const float w = nu[k] > 0 ? curve_weight(tok[k], si.len, p.a, p.b) : 0.f;
+    const float w = nu[k] > 0 ? curve_weight(tok[k], si.len, si.a, si.b) : 0.f;
     out[k] = w > 0.f ? log2f(w) - (acc[k].x + log2f(acc[k].y)) : -INFINITY;
   }
 }
@@ -337,9 +359,10 @@ __device__ inline void plan_prologue(PassArgs& p, const PassArgs& pa, const Host
     p.seqs = lp->seqs;
     p.e1 = lp->e1;
     p.e2 = lp->e2;
-    if (p1) {
+    if (p1 || pa.lse) {
       // this call's device status word, and zero scores for sequences
-      // without an active row (the planner kernel's duties)
+      // without an active row (the planner kernel's duties), in the first
+      // pass the call runs
       if (blockIdx.x == 0 && threadIdx.x == 0) *pa.status = lp->hdr.status;
       if (lp->hdr.status == 0) {
         const int64_t stride = (int64_t)gridDim.x * blockDim.x;

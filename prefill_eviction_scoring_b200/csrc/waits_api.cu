@@ -122,7 +122,9 @@ uint32_t* status_word(void* ws, size_t bytes) {
 }
 
 waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, float a,
-                           int32_t b, float* scores, void* ws, cudaStream_t st) {
+                           int32_t b, float* scores, void* ws, cudaStream_t st,
+                           const float* lse = nullptr, const float* seq_a = nullptr,
+                           const int32_t* seq_b = nullptr) {
   const Layout L = layout_of(s);
   uint8_t* base = static_cast<uint8_t*>(ws);
   const int grid = grid_size();
@@ -138,6 +140,8 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   pa.tokq = tokens_per_qtile(pa.G);
   pa.a = a;
   pa.b = b;
+  pa.seq_a = seq_a;
+  pa.seq_b = seq_b;
   pa.grid = grid;
   pa.hdr = reinterpret_cast<PlanHeader*>(base + L.header);
   pa.seqs = reinterpret_cast<SeqInfo*>(base + L.seqs);
@@ -149,7 +153,8 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   pa.max_u1 = L.max_u1;
   pa.max_u2 = L.max_u2;
   pa.scores = scores;
-  const bool local = local_plan_fits(s, a, b);
+  // routed calls plan on the device from the per-sequence parameters
+  const bool local = !seq_a && local_plan_fits(s, a, b);
   cudaError_t err = cudaSuccess;
   if (!local) {
     err = launch_plan(pa, st);
@@ -178,6 +183,7 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   p.scores = scores;
   p.status = &pa.hdr->status;
   p.local_plan = local ? 1 : 0;
+  p.lse = lse;
   p.wait_ns = wait_limit_ns();
   p.withhold_mma = withhold_mma() ? 1 : 0;
   p.cu = s->cu_seqlens;
@@ -277,6 +283,42 @@ waits_status waits_score(const waits_shape* shape, const void* Q, const void* K,
   if (st == WAITS_OK) st = check_ws(shape, workspace, workspace_bytes);
   if (st != WAITS_OK) return st;
   return enqueue_score(shape, Q, K, a, b, scores, workspace, static_cast<cudaStream_t>(stream));
+}
+
+waits_status waits_score_with_lse(const waits_shape* shape, const void* Q, const void* K,
+                                  const float* lse, float a, int32_t b, float* scores,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  waits_status st = check_shape(shape);
+  if (st == WAITS_OK) st = check_score_args(shape, Q, K, a, b, scores);
+  if (st == WAITS_OK && (!lse || !aligned(lse, 4))) st = WAITS_ERR_ARG;
+  if (st == WAITS_OK) st = check_ws(shape, workspace, workspace_bytes);
+  if (st != WAITS_OK) return st;
+  return enqueue_score(shape, Q, K, a, b, scores, workspace, static_cast<cudaStream_t>(stream),
+                       lse);
+}
+
+waits_status waits_score_routed(const waits_shape* shape, const void* Q, const void* K,
+                                const float* a, const int32_t* b, float* scores,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  waits_status st = check_shape(shape);
+  if (st == WAITS_OK) st = check_score_args(shape, Q, K, 0.0f, 0, scores);
+  if (st == WAITS_OK && (!a || !b || !aligned(a, 4) || !aligned(b, 4))) st = WAITS_ERR_ARG;
+  if (st == WAITS_OK) st = check_ws(shape, workspace, workspace_bytes);
+  if (st != WAITS_OK) return st;
+  return enqueue_score(shape, Q, K, 0.0f, 0, scores, workspace,
+                       static_cast<cudaStream_t>(stream), nullptr, a, b);
+}
+
+waits_status waits_compress_routed(const waits_shape* shape, const void* Q, const void* K,
+                                   const void* V, const float* a, const int32_t* b, int32_t R,
+                                   int32_t B, float* scores, int32_t* idx, int32_t* kept_len,
+                                   void* K_out, void* V_out, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  waits_status st = waits_score_routed(shape, Q, K, a, b, scores, workspace, workspace_bytes,
+                                       stream);
+  if (st != WAITS_OK) return st;
+  return waits_select_compact(shape, scores, K, V, R, B, idx, kept_len, K_out, V_out, workspace,
+                              workspace_bytes, stream);
 }
 
 waits_status waits_select(const waits_shape* shape, const float* scores, int32_t R, int32_t B,

@@ -39,7 +39,9 @@ struct SeqInfo {
   int32_t nkt;     // K tiles covering keys [0, N)
   int32_t e1;      // first pass-1 entry of this sequence
   int32_t e2;      // first pass-2 entry of this sequence
-  int32_t pad;
+  int32_t b;       // this sequence's forgetting-curve window and slope
+  float a;
+  int32_t pad[3];  // 48 bytes: arrays of entries after it stay 16-byte aligned
 };
 
 // An entry is one (sequence, KV head, stationary group) with a contiguous
@@ -209,6 +211,9 @@ struct PlanArgs {
   int nseq, T, max_seqlen, Hq, Hkv, G, tokq;
   float a;
   int b;
+  // per-sequence curve parameters (DEVICE [nseq]; routed calls), else null
+  const float* seq_a;
+  const int32_t* seq_b;
   int grid;
   PlanHeader* hdr;
   SeqInfo* seqs;
@@ -242,6 +247,9 @@ struct PassArgs {
   int host_plan;
   const int32_t* cu;
   int nseq, max_seqlen;
+  // natural-log row LSE [Hq, T] given by the caller (waits_score_with_lse):
+  // pass 1 is not run and pass 2 takes its row biases from it; else null
+  const float* lse;
   // limit of every bounded wait in the main loops (ns); testing aid: with
   // withhold_mma the MMA warp issues nothing, so those waits run out
   uint64_t wait_ns;

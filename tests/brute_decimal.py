@@ -45,3 +45,26 @@ def brute_scores(Q, K, cu_seqlens, a, b, prec=40):
                     for k in range(q + 1):
                         s[g][lo + k] += w * ex[k] / z
         return s
+
+
+def brute_lse(Q, K, cu_seqlens, prec=40):
+    """Natural-log row LSE [Hq][T] of the causal attention, in decimal."""
+    T = len(Q)
+    Hq = len(Q[0]) if T else 0
+    Hkv = len(K[0]) if T else 0
+    d = len(Q[0][0]) if T else 0
+    G = Hq // Hkv if Hkv else 1
+    with localcontext() as ctx:
+        ctx.prec = prec
+        out = [[Decimal(0) for _ in range(T)] for _ in range(Hq)]
+        root_d = Decimal(d).sqrt() if d else Decimal(1)
+        for i in range(len(cu_seqlens) - 1):
+            lo, hi = int(cu_seqlens[i]), int(cu_seqlens[i + 1])
+            for h in range(Hq):
+                g = h // G
+                for q in range(hi - lo):
+                    logits = [sum(Decimal(float(Q[lo + q][h][j])) * Decimal(float(K[lo + k][g][j]))
+                                  for j in range(d)) / root_d for k in range(q + 1)]
+                    m = max(logits)
+                    out[h][lo + q] = m + sum((x - m).exp() for x in logits).ln()
+        return out

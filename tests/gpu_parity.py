@@ -25,6 +25,16 @@ def run_gpu(lay, a, b, R, B, canary=True):
         nid = c.idx.numel()
         bigi = torch.full((nid + 2 * pad,), -777, dtype=torch.int32, device="cuda")
         c.idx = bigi[pad:pad + nid].view_as(c.idx)
+        nk = c.kept_len.numel()
+        bigk = torch.full((nk + 2 * pad,), -555, dtype=torch.int32, device="cuda")
+        c.kept_len = bigk[pad:pad + nk]
+        # K_out / V_out: guard rows of 16-byte vectors (the kernels write whole rows)
+        no = c.K_out.numel()
+        gpad = 8 * d
+        bigo = [torch.full((no + 2 * gpad,), 7.5, dtype=torch.bfloat16, device="cuda")
+                for _ in range(2)]
+        c.K_out = bigo[0][gpad:gpad + no].view_as(c.K_out)
+        c.V_out = bigo[1][gpad:gpad + no].view_as(c.V_out)
     Ko, Vo, idx, kept, s = c(lay.Q, lay.K, lay.V, a, b, R)
     torch.cuda.synchronize()
     status = c.device_status()
@@ -32,6 +42,9 @@ def run_gpu(lay, a, b, R, B, canary=True):
     if canary:
         assert torch.all(big[:pad] == -7.0) and torch.all(big[pad + Hkv * T:] == -7.0)
         assert torch.all(bigi[:pad] == -777) and torch.all(bigi[pad + nid:] == -777)
+        assert torch.all(bigk[:pad] == -555) and torch.all(bigk[pad + nk:] == -555)
+        for t in bigo:
+            assert torch.all(t[:gpad] == 7.5) and torch.all(t[gpad + no:] == 7.5)
     return dict(scores=s.double().cpu().numpy(), idx=idx.cpu().numpy(),
                 kept=kept.cpu().numpy(), Ko=Ko.cpu().view(torch.int16).numpy(),
                 Vo=Vo.cpu().view(torch.int16).numpy(), raw_scores=s.clone())

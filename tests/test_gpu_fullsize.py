@@ -24,19 +24,30 @@ def _group_ref(lay, g, a, b):
     return oracle.score(Q, K, lay.cu_seqlens.cpu().numpy(), a, b)[0]
 
 
-@pytest.mark.parametrize("layer,B", [(0, 2048), (0, 512), (31, 128)])
-def test_llama8b_full(layer, B):
+def _group_tail_ref(lay, g, a, b, W):
+    """Oracle scores of KV head g from the last W rows of each sequence:
+    exact for the last W keys (a key is seen only by rows at or after it)."""
+    Hq, Hkv = lay.Q.shape[1], lay.K.shape[1]
+    G = Hq // Hkv
+    Q = wl.to_numpy64(lay.Q[:, g * G:(g + 1) * G])
+    K = wl.to_numpy64(lay.K[:, g:g + 1])
+    return oracle.score(Q, K, lay.cu_seqlens.cpu().numpy(), a, b, last=W)[0]
+
+
+@pytest.mark.parametrize("layer,B,heads", [(0, 2048, tuple(range(8))), (0, 512, (0, 5)),
+                                           (31, 128, (2, 7))])
+def test_llama8b_full(layer, B, heads):
     spec = wl.CONFIGS["llama8b"]
     lay = wl.make_layer("llama8b", layer=layer, device="cuda")
     a, b = spec.actions[0]
     gpu = run_gpu(lay, a, b, spec.recent, B)
     cu = lay.cu_seqlens.cpu().numpy()
     ref = np.zeros_like(gpu["scores"])
-    for g in (0, 5):
+    for g in heads:
         ref[g] = _group_ref(lay, g, a, b)
         assert_scores_close(gpu["scores"][g:g + 1], ref[g:g + 1])
     # selection / compaction for the checked heads
-    for g in (0, 5):
+    for g in heads:
         sub_idx = gpu["idx"][:, g:g + 1]
         assert_selection(sub_idx, gpu["kept"], ref[g:g + 1], gpu["scores"][g:g + 1], cu,
                          spec.recent, B)
@@ -108,3 +119,28 @@ def test_llama8b_dense_properties():
     np.testing.assert_array_equal(gpu["idx"], self_idx)
     np.testing.assert_array_equal(gpu["kept"], self_kept)
     assert_compaction(lay, gpu, B)
+
+
+def test_long_full_tail_exact():
+    """The 131072-token layer (a = 0.01, b = 128: some 9000 active rows):
+    the last 1024 keys of two KV heads against the oracle, element by
+    element; they depend only on the last 1024 rows."""
+    spec = wl.CONFIGS["long"]
+    lay = wl.make_layer("long", device="cuda")
+    a, b = spec.actions[0]
+    gpu = run_gpu(lay, a, b, spec.recent, spec.budgets[0])
+    N, W = lay.total_tokens, 1024
+    for g in (1, 6):
+        ref = _group_tail_ref(lay, g, a, b, W)
+        assert_scores_close(gpu["scores"][g:g + 1, N - W:], ref[None, N - W:])
+
+
+def test_llama8b_dense_tail_exact():
+    """The 8B layer with a = 0 (every row active): the last 2048 keys of two
+    KV heads against the oracle, element by element."""
+    lay = wl.make_layer("llama8b", layer=7, device="cuda")
+    gpu = run_gpu(lay, 0.0, 16, 16, 2048)
+    N, W = lay.total_tokens, 2048
+    for g in (0, 4):
+        ref = _group_tail_ref(lay, g, 0.0, 16, W)
+        assert_scores_close(gpu["scores"][g:g + 1, N - W:], ref[None, N - W:])

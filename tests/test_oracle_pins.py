@@ -100,3 +100,19 @@ def test_fp32_zero_weight_rows_are_negligible(N, a, b):
     # and the kept rows form a suffix of the sequence
     act = np.nonzero(w32 != 0)[0]
     assert len(act) == 0 or np.all(act == np.arange(act[0], N))
+
+
+def test_last_rows_give_the_exact_tail():
+    """Key k is seen only by rows q >= k: summing the last W rows gives the
+    exact scores of the last W keys of every sequence, and never more than
+    the full scores elsewhere."""
+    Q = pins._rand((210, 4, 8), 51)
+    K = pins._rand((210, 2, 8), 52)
+    cu = np.array([0, 130, 210])
+    for a, b in ((0.0, 4), (0.05, 20), (1.0, 3)):
+        full = oracle.score(Q, K, cu, a, b)
+        part = oracle.score(Q, K, cu, a, b, last=25)
+        tail = np.r_[105:130, 185:210]
+        np.testing.assert_array_equal(part[:, tail], full[:, tail])
+        assert np.all(part <= full * (1 + 1e-12))
+        assert np.all(part[:, :100] < full[:, :100]) or a > 0.5
