@@ -98,6 +98,10 @@ def parse(argv=None):
                    help="B (default: 2048 for llama8b, the workload's budget otherwise); "
                         "for llama8b, --budget all sweeps 128, 512 and 2048")
     p.add_argument("--layers", type=int, default=None)
+    p.add_argument("--parallel", choices=["layers", "heads"], default="layers",
+                   help="multi-GPU split: every rank its own layers (weak scaling, default) "
+                        "or every rank its share of the KV heads of the same layers "
+                        "(tensor-parallel style, strong scaling)")
     p.add_argument("--e2e-layers", type=int, default=4)
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -108,6 +112,14 @@ def parse(argv=None):
     if rest:
         p.error(f"unknown arguments {rest}")
     return args
+
+
+def head_shard(rank: int, world: int, Hkv: int) -> Tuple[int, int]:
+    """KV heads [g0, g1) of ``rank`` when ``world`` ranks split a layer's
+    ``Hkv`` heads contiguously (ranks past Hkv own none)."""
+    g0 = rank * Hkv // world if world <= Hkv else min(rank, Hkv)
+    g1 = (rank + 1) * Hkv // world if world <= Hkv else min(rank + 1, Hkv)
+    return g0, g1
 
 
 # ------------------------------------------------------------ arithmetic ---
@@ -508,6 +520,76 @@ def config_dict(case: Case, lens, spec, L, flushed):
 
 
 # ------------------------------------------------------------------ ours ---
+def run_heads_case(args, D, lib, case: Case):
+    """Every rank compresses its contiguous share of the KV heads of the same
+    layers (waits_compress_heads, in place); value = the layers' tokens per
+    second of the slowest rank (strong scaling)."""
+    dev = torch.device("cuda", D.local)
+    spec = wl.CONFIGS[case.config]
+    L, a, b, R, B = case.layers, case.a, case.b, case.R, case.B
+    layers = [wl.make_layer(case.config, layer=i, device=dev) for i in range(L)]
+    lay0 = layers[0]
+    T, Hq, d = lay0.Q.shape
+    Hkv = lay0.K.shape[1]
+    g0, g1 = head_shard(D.rank, D.world, Hkv)
+    Hs, nseq = g1 - g0, len(lay0.lens)
+    shape = api.make_shape(lay0.cu_seqlens, T, lay0.max_seqlen, Hq, Hkv, d)
+    ws_bytes = api.workspace_bytes(shape)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    scores = torch.empty((max(Hs, 1), T), dtype=torch.float32, device=dev)
+    idx = torch.empty((nseq, max(Hs, 1), B), dtype=torch.int32, device=dev)
+    kept = torch.empty((nseq,), dtype=torch.int32, device=dev)
+    Ko = torch.empty((nseq, max(Hs, 1), B, d), dtype=torch.bfloat16, device=dev)
+    Vo = torch.empty_like(Ko)
+    sp = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+    def step():
+        if Hs == 0:
+            return
+        for l in layers:
+            _lib.check("waits_compress_heads", lib.waits_compress_heads(
+                ctypes.byref(shape), g0, g1, l.Q.data_ptr(), l.K.data_ptr(), l.V.data_ptr(), a,
+                b, R, B, scores.data_ptr(), idx.data_ptr(), kept.data_ptr(), Ko.data_ptr(),
+                Vo.data_ptr(), ws.data_ptr(), ws_bytes, sp))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(D.local)
+    D.barrier()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    D.barrier()
+    ms = D.max(e0.elapsed_time(e1) / args.steps)
+    if D.rank == 0:
+        pk, pk_kind = peaks()
+        sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+        # the slowest rank against its own share of the work (the whole
+        # layer's work split over the ranks that own heads)
+        owners = min(D.world, Hkv)
+        _, other = rooflines(lay0.lens, Hq, Hkv, d, a, b, B, ms / L, 0.0, ms / L, pk, sm_count,
+                             peak_kind=pk_kind)
+        layer_roof = dict(other[0])
+        layer_roof["roofline_us"] = round(layer_roof["roofline_us"] / owners, 2)
+        layer_roof["frac"] = round(layer_roof["roofline_us"] / (ms / L * 1e3), 4)
+        cfg = config_dict(case, lay0.lens, spec, L, False)
+        cfg["parallelism"] = f"heads: {D.world} ranks split the {Hkv} KV heads of every layer"
+        out = {"metric": METRIC, "value": L * sum(lay0.lens) / (ms / 1e3), "unit": UNIT,
+               "n_gpus": D.world, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+               "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+               "roofline": layer_roof, "clocks": clk,
+               "gpu_launches": (score_kernels(lib, shape, a, b) + KERNELS_OUTSIDE_SCORE) * L *
+               args.steps, "per_layer_us": {"layer": round(ms / L * 1e3, 2)}}
+        print(json.dumps(out), flush=True)
+
+
 def run_case(args, D, lib, case: Case, headline: bool):
     dev = torch.device("cuda", D.local)
     spec = wl.CONFIGS[case.config]
@@ -696,6 +778,9 @@ def run_ours(args):
     D.init()
     lib = _lib.load()
     for case in selected_cases(args):
+        if args.parallel == "heads":
+            run_heads_case(args, D, lib, case)
+            continue
         headline = (case.name == "llama8b" and case.B == 2048 and args.config == "llama8b")
         run_case(args, D, lib, case, headline)
     D.close()

@@ -228,6 +228,30 @@ waits_status waits_compress(const waits_shape* shape, const void* Q, const void*
                             void* K_out, void* V_out, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/*
+ * waits_compress for the KV heads [kv_head_begin, kv_head_end) of a layer,
+ * reading the layer's own Q, K and V in place: a tensor-parallel rank that
+ * owns those heads scores, selects and compacts exactly them (every KV head,
+ * with its query heads, is independent of the others; no exchange between
+ * ranks is needed, since a rank's compacted cache is what its decode reads).
+ *   shape            the whole layer (num_q_heads, num_kv_heads of the tensors)
+ *   Q, K, V          the whole layer's tensors, as for waits_compress
+ *   scores           fp32 [Hs, T], Hs = kv_head_end - kv_head_begin: row i
+ *                    is KV head kv_head_begin + i
+ *   idx, kept_len    [nseq, Hs, B], [nseq]
+ *   K_out, V_out     bf16 [nseq, Hs, B, d]
+ *   workspace        >= waits_workspace_size() of the layer (a range needs no more)
+ * The results equal the rows of a whole-layer call for those heads, up to
+ * the fp32 rounding of sums whose order depends on the work split.
+ * Errors: as waits_compress, plus ARG for an empty or out-of-range range.
+ */
+waits_status waits_compress_heads(const waits_shape* shape, int32_t kv_head_begin,
+                                  int32_t kv_head_end, const void* Q, const void* K,
+                                  const void* V, float a, int32_t b, int32_t R, int32_t B,
+                                  float* scores, int32_t* idx, int32_t* kept_len, void* K_out,
+                                  void* V_out, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
 /* Device buffers that waits_compress_host stages through (caller-owned). */
 typedef struct waits_device_buffers {
   void* Q;          /* bf16 [T, Hq, d]  */
@@ -327,6 +351,39 @@ waits_status waits_read_static_status(void* stream, uint32_t* status_bits);
 waits_status waits_read_device_status(const void* workspace,
                                       size_t workspace_bytes, void* stream,
                                       uint32_t* status_bits);
+
+/*
+ * Bytes of device workspace waits_decode_attention needs.  Host-only.
+ * Errors: ARG (bytes NULL), SHAPE, UNSUPPORTED (head_dim not 64 or 128).
+ */
+waits_status waits_decode_workspace_size(int32_t nseq, int32_t num_q_heads, int32_t head_dim,
+                                         int32_t capacity, size_t* bytes);
+
+/*
+ * One decode step of attention over the compacted cache: what the model
+ * runs after prefill compression (README Quickstart: model.generate after
+ * init_cache).  For sequence s and query head h, KV head g = h / G:
+ *   out[s, h] = sum_{j < cache_len[s]} softmax_j(q[s, h] . K_cache[s, g, j] / sqrt(d))
+ *               * V_cache[s, g, j]
+ *   lse[s, h] = natural log of that softmax's normaliser (-inf, and out = 0,
+ *               for an empty cache)
+ *   q          DEVICE bf16 [nseq, Hq, d], 16-byte aligned
+ *   K_cache, V_cache  DEVICE bf16 [nseq, Hkv, capacity, d] (waits_compress's
+ *               K_out, V_out with capacity = B, or any cache of that layout;
+ *               slots past cache_len[s] are not read)
+ *   cache_len  DEVICE int32 [nseq]: valid slots (kept_len, plus any decoded
+ *               tokens the caller appended); clamped to [0, capacity]
+ *   out        DEVICE fp32 [nseq, Hq, d];  lse  DEVICE fp32 [nseq, Hq] or NULL
+ *   workspace  >= waits_decode_workspace_size() bytes, 16-byte aligned
+ * Two kernels on `stream` (per 256 cache slots, then the merge).  Hq / Hkv
+ * at most 16.
+ * Errors: ARG, SHAPE, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+waits_status waits_decode_attention(int32_t nseq, int32_t num_q_heads, int32_t num_kv_heads,
+                                    int32_t head_dim, int32_t capacity, const void* q,
+                                    const void* K_cache, const void* V_cache,
+                                    const int32_t* cache_len, float* out, float* lse,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Testing aid, no counterpart on the WAITS pages: y[i] = the scorer's

@@ -23,4 +23,5 @@ from .waits_oracle import (  # noqa: F401
     select,
     compact,
     compress,
+    decode_attention,
 )

@@ -201,6 +201,40 @@ def compact(K, V, cu_seqlens, idx, kept_len, B):
     return Ko, Vo
 
 
+def decode_attention(q, K_cache, V_cache, cache_len):
+    """One decode step of attention over the compacted cache, fp64.
+
+    After prefill the model generates from the compressed cache (WAITS
+    README, Quickstart: ``model.generate`` after ``init_cache``).  For
+    sequence s and query head h (KV head g = h // G):
+    ``o[s, h] = sum_{j < cache_len[s]} softmax_j(q[s, h] . K[s, g, j] / sqrt(d)) V[s, g, j]``
+    and ``lse[s, h]`` = the natural-log normaliser of that softmax.
+
+    q ``[nseq, Hq, d]``, K_cache and V_cache ``[nseq, Hkv, C, d]`` (C slots,
+    the first cache_len[s] valid), cache_len ``[nseq]``.  A sequence with an
+    empty cache gets o = 0 and lse = -inf.  Returns ``(o, lse)``.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    Kc = np.asarray(K_cache, dtype=np.float64)
+    Vc = np.asarray(V_cache, dtype=np.float64)
+    nseq, Hq, d = q.shape
+    Hkv = Kc.shape[1]
+    G = Hq // Hkv
+    o = np.zeros((nseq, Hq, d))
+    lse = np.full((nseq, Hq), -np.inf)
+    for s in range(nseq):
+        n = int(cache_len[s])
+        if n <= 0:
+            continue
+        for h in range(Hq):
+            L = Kc[s, h // G, :n] @ q[s, h] / np.sqrt(float(d))
+            m = L.max()
+            e = np.exp(L - m)
+            o[s, h] = (e[:, None] * Vc[s, h // G, :n]).sum(axis=0) / e.sum()
+            lse[s, h] = m + np.log(e.sum())
+    return o, lse
+
+
 def compress(Q, K, V, cu_seqlens, a, b, R, B, *, K_bits=None, V_bits=None):
     """score -> select -> compact, as one call.
 

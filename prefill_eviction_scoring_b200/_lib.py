@@ -60,6 +60,8 @@ SIGNATURES = {
     "waits_score": (_I, [_PSHAPE, _P, _P, _F, _I, _P, _P, _SZ, _P]),
     "waits_score_with_lse": (_I, [_PSHAPE, _P, _P, _P, _F, _I, _P, _P, _SZ, _P]),
     "waits_score_routed": (_I, [_PSHAPE, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "waits_compress_heads": (_I, [_PSHAPE, _I, _I, _P, _P, _P, _F, _I, _I, _I, _P, _P, _P,
+                                  _P, _P, _P, _SZ, _P]),
     "waits_compress_routed": (_I, [_PSHAPE, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P,
                                    _P, _SZ, _P]),
     "waits_select": (_I, [_PSHAPE, _P, _I, _I, _P, _P, _P, _SZ, _P]),
@@ -75,6 +77,8 @@ SIGNATURES = {
     "waits_score_static": (_I, [_PSHAPE, _P, _P, _F, _I, _P, _P]),
     "waits_read_static_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "waits_test_exp2_poly": (_I, [_P, _P, ctypes.c_int64, _P]),
+    "waits_decode_workspace_size": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),
+    "waits_decode_attention": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "waits_score_kernels": (_I, [_PSHAPE, _F, _I, ctypes.POINTER(ctypes.c_int32)]),
     "waits_select_compact": (_I, [_PSHAPE, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
 }

@@ -170,6 +170,70 @@ def score(Q: torch.Tensor, K: torch.Tensor, cu_seqlens: torch.Tensor, *,
     return c.score(Q, K, sigmoid_a, window)
 
 
+def compress_heads(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                   kv_heads: Tuple[int, int], *, sigmoid_a: float, window: int,
+                   recent_budget: int, budget: int, max_seqlen: Optional[int] = None):
+    """``waits_compress_heads``: score, select and compact the KV heads
+    ``[kv_heads[0], kv_heads[1])`` of the layer, reading ``q, k, v`` in place
+    (a tensor-parallel rank's share).  Returns ``(K_out, V_out, idx,
+    kept_len, scores)`` for those heads only."""
+    _need_cuda("q", q, torch.bfloat16)
+    _need_cuda("k", k, torch.bfloat16)
+    _need_cuda("v", v, torch.bfloat16)
+    _need_cuda("cu_seqlens", cu_seqlens, torch.int32)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    g0, g1 = int(kv_heads[0]), int(kv_heads[1])
+    Hs = g1 - g0
+    nseq = cu_seqlens.numel() - 1
+    dev = q.device
+    lib = _lib.load()
+    shape = make_shape(cu_seqlens, T, _max_seqlen(cu_seqlens, max_seqlen), Hq, Hkv, d)
+    ws_bytes = workspace_bytes(shape)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    scores = torch.empty((max(Hs, 0), T), dtype=torch.float32, device=dev)
+    idx = torch.empty((nseq, max(Hs, 0), budget), dtype=torch.int32, device=dev)
+    kept = torch.empty((nseq,), dtype=torch.int32, device=dev)
+    Ko = torch.empty((nseq, max(Hs, 0), budget, d), dtype=torch.bfloat16, device=dev)
+    Vo = torch.empty_like(Ko)
+    st = lib.waits_compress_heads(ctypes.byref(shape), g0, g1, _ptr(q), _ptr(k), _ptr(v),
+                                  float(sigmoid_a), int(window), int(recent_budget), int(budget),
+                                  _ptr(scores), _ptr(idx), _ptr(kept), _ptr(Ko), _ptr(Vo),
+                                  _ptr(ws), ws_bytes, _stream(dev))
+    _lib.check("waits_compress_heads", st)
+    return Ko, Vo, idx, kept, scores
+
+
+def decode_attention(q: torch.Tensor, K_cache: torch.Tensor, V_cache: torch.Tensor,
+                     cache_len: torch.Tensor, with_lse: bool = False):
+    """One decode step over the compacted cache (``waits_decode_attention``).
+
+    ``q`` bf16 ``[nseq, Hq, d]``; ``K_cache``, ``V_cache`` bf16 ``[nseq, Hkv,
+    C, d]`` (e.g. waits_compress's outputs); ``cache_len`` int32 ``[nseq]``.
+    Returns fp32 ``[nseq, Hq, d]`` (and the fp32 ``[nseq, Hq]`` row LSE).
+    """
+    _need_cuda("q", q, torch.bfloat16)
+    _need_cuda("K_cache", K_cache, torch.bfloat16)
+    _need_cuda("V_cache", V_cache, torch.bfloat16)
+    _need_cuda("cache_len", cache_len, torch.int32)
+    nseq, Hq, d = q.shape
+    Hkv, C = K_cache.shape[1], K_cache.shape[2]
+    if tuple(K_cache.shape) != (nseq, Hkv, C, d) or V_cache.shape != K_cache.shape:
+        raise ValueError("caches must be [nseq, Hkv, C, d] like q's [nseq, Hq, d]")
+    lib = _lib.load()
+    n = ctypes.c_size_t(0)
+    _lib.check("waits_decode_workspace_size",
+               lib.waits_decode_workspace_size(nseq, Hq, d, C, ctypes.byref(n)))
+    ws = torch.empty(max(n.value, 16), dtype=torch.uint8, device=q.device)
+    out = torch.empty((nseq, Hq, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((nseq, Hq), dtype=torch.float32, device=q.device) if with_lse else None
+    st = lib.waits_decode_attention(nseq, Hq, Hkv, d, C, _ptr(q), _ptr(K_cache), _ptr(V_cache),
+                                    _ptr(cache_len), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                    _stream(q.device))
+    _lib.check("waits_decode_attention", st)
+    return (out, lse) if with_lse else out
+
+
 def score_with_lse(Q: torch.Tensor, K: torch.Tensor, cu_seqlens: torch.Tensor,
                    lse: torch.Tensor, *, sigmoid_a: float, window: int,
                    max_seqlen: Optional[int] = None) -> torch.Tensor:

@@ -15,7 +15,8 @@ template <int LOG_CPR>
 __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
     const uint4* __restrict__ K, const uint4* __restrict__ V, const int32_t* __restrict__ cu,
     const int32_t* __restrict__ idx, const int32_t* __restrict__ kept_len, int Hkv, int B,
-    uint32_t total, uint4* __restrict__ Ko, uint4* __restrict__ Vo, uint32_t* status) {
+    int row_heads, uint32_t total, uint4* __restrict__ Ko, uint4* __restrict__ Vo,
+    uint32_t* status) {
   constexpr int kCpr = 1 << LOG_CPR;                 // 16-byte vectors per row (d / 8)
   pdl_allow_next();
   pdl_wait();
@@ -35,7 +36,7 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
   if (j < kl) {
     const int N = hi - lo;
     if (k >= 0 && k < N) {
-      const size_t src = ((size_t)(lo + k) * Hkv + g) * kCpr + c;
+      const size_t src = ((size_t)(lo + k) * row_heads + g) * kCpr + c;
       kv = __ldg(K + src);
       vv = __ldg(V + src);
     } else if (status && c == 0) {
@@ -51,7 +52,8 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
 cudaError_t launch_compact(const uint16_t* K, const uint16_t* V, const int32_t* cu,
                            const int32_t* idx, const int32_t* kept_len, int nseq, int Hkv,
                            int d, int B, uint16_t* Ko, uint16_t* Vo, uint32_t* status,
-                           cudaStream_t s) {
+                           cudaStream_t s, int kv_row_heads) {
+  const int rh = kv_row_heads > 0 ? kv_row_heads : Hkv;
   const int64_t total = (int64_t)nseq * Hkv * B * (d / 8);
   if (total >= 0x7fffff00LL) return cudaErrorInvalidValue;
   const unsigned blocks = (unsigned)((total + kCompactThreads - 1) / kCompactThreads);
@@ -61,9 +63,9 @@ cudaError_t launch_compact(const uint16_t* K, const uint16_t* V, const int32_t* 
   uint4* vo = reinterpret_cast<uint4*>(Vo);
   if (d == 128)
     return launch_pdl(compact_kernel<4>, dim3(blocks), dim3(kCompactThreads), 0, s, k4, v4, cu,
-                      idx, kept_len, Hkv, B, (uint32_t)total, ko, vo, status);
+                      idx, kept_len, Hkv, B, rh, (uint32_t)total, ko, vo, status);
   return launch_pdl(compact_kernel<3>, dim3(blocks), dim3(kCompactThreads), 0, s, k4, v4, cu, idx,
-                    kept_len, Hkv, B, (uint32_t)total, ko, vo, status);
+                    kept_len, Hkv, B, rh, (uint32_t)total, ko, vo, status);
 }
 
 }  // namespace waits

@@ -492,8 +492,8 @@ static_assert(sizeof(HostPlan) + 2 * sizeof(CUtensorMap) + sizeof(PassArgs) + 64
 template <int D>
 cudaError_t launch_sparse_d(const PassArgs& a, const HostPlan& hp, int grid, cudaStream_t st) {
   CUtensorMap mq, mk;
-  if (!make_map(&mq, a.Q, a.T, a.Hq, D, a.G, a.tokq) ||
-      !make_map(&mk, a.K, a.T, a.Hkv, D, 1, kTile))
+  if (!make_map(&mq, a.Q, a.T, a.Hq, a.q_row_heads, D, a.G, a.tokq) ||
+      !make_map(&mk, a.K, a.T, a.Hkv, a.kv_row_heads, D, 1, kTile))
     return cudaErrorInvalidValue;
   const size_t smem1 = sparse_smem<D, 1>(), smem2 = sparse_smem<D, 2>();
   cudaError_t err;

@@ -398,11 +398,14 @@ inline EncodeTiledFn encode_fn() {
 }
 
 // 3-D view [T][heads][d] of a packed bf16 tensor; box = 64 x box_h x box_t.
-inline bool make_map(CUtensorMap* m, const void* base, int T, int heads, int d, int box_h, int box_t) {
+inline bool make_map(CUtensorMap* m, const void* base, int T, int heads, int row_heads, int d,
+                     int box_h, int box_t) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  // `heads` heads of each token row are addressed; a row holds `row_heads`
+  // (more when the call covers a range of the layer's heads)
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)T};
-  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)row_heads * d * 2};
   const cuuint32_t box[3] = {64u, (cuuint32_t)box_h, (cuuint32_t)box_t};
   const cuuint32_t elem[3] = {1u, 1u, 1u};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,

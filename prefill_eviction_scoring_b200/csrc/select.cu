@@ -71,6 +71,7 @@ struct KVCopy {
   uint4* Ko;
   uint4* Vo;
   int log_cpr;
+  int row_heads;   // heads per token row of K and V in memory
 };
 
 // Output rows [r0, r1) of (sequence s, KV head g): slot j gets source
@@ -106,7 +107,7 @@ __device__ inline void copy_rows(const KVCopy& c, int Hkv, int B, int s, int g, 
         const int src = src_of(j);
         dst[u] = ((out0 + j) << c.log_cpr) + col;
         if (src >= 0) {
-          const size_t from = ((((size_t)lo + src) * Hkv + g) << c.log_cpr) + col;
+          const size_t from = ((((size_t)lo + src) * c.row_heads + g) << c.log_cpr) + col;
           kx[u] = __ldg(K + from);
           vx[u] = ld_global_v4(V + from);
         }
@@ -493,12 +494,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int T, int Hkv,
                           int R, int B, int32_t* idx, int32_t* kept_len, uint32_t* status,
                           cudaStream_t s, const uint16_t* K, const uint16_t* V, int d,
-                          uint16_t* Ko, uint16_t* Vo) {
+                          uint16_t* Ko, uint16_t* Vo, int kv_row_heads) {
   const int64_t grid = (int64_t)nseq * Hkv * kC;
   if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
   const int dyn = kStageGroups * (int)sizeof(uint4) + (int)sizeof(SelSmem);
   KVCopy kv{reinterpret_cast<const uint4*>(K), reinterpret_cast<const uint4*>(V),
-            reinterpret_cast<uint4*>(Ko), reinterpret_cast<uint4*>(Vo), d == 128 ? 4 : 3};
+            reinterpret_cast<uint4*>(Ko), reinterpret_cast<uint4*>(Vo), d == 128 ? 4 : 3,
+            kv_row_heads > 0 ? kv_row_heads : Hkv};
   auto kernel = K ? select_kernel<true> : select_kernel<false>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
   if (err != cudaSuccess) return err;

@@ -124,7 +124,8 @@ uint32_t* status_word(void* ws, size_t bytes) {
 waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, float a,
                            int32_t b, float* scores, void* ws, cudaStream_t st,
                            const float* lse = nullptr, const float* seq_a = nullptr,
-                           const int32_t* seq_b = nullptr) {
+                           const int32_t* seq_b = nullptr, int q_row_heads = 0,
+                           int kv_row_heads = 0) {
   const Layout L = layout_of(s);
   uint8_t* base = static_cast<uint8_t*>(ws);
   const int grid = grid_size();
@@ -167,6 +168,8 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
   p.T = s->total_tokens;
   p.Hq = s->num_q_heads;
   p.Hkv = s->num_kv_heads;
+  p.q_row_heads = q_row_heads > 0 ? q_row_heads : s->num_q_heads;
+  p.kv_row_heads = kv_row_heads > 0 ? kv_row_heads : s->num_kv_heads;
   p.G = pa.G;
   p.tokq = pa.tokq;
   p.d = s->head_dim;
@@ -373,6 +376,43 @@ waits_status waits_compress(const waits_shape* shape, const void* Q, const void*
   return WAITS_OK;
 }
 
+waits_status waits_compress_heads(const waits_shape* shape, int32_t kv_head_begin,
+                                  int32_t kv_head_end, const void* Q, const void* K,
+                                  const void* V, float a, int32_t b, int32_t R, int32_t B,
+                                  float* scores, int32_t* idx, int32_t* kept_len, void* K_out,
+                                  void* V_out, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  waits_status st = check_shape(shape);
+  if (st != WAITS_OK) return st;
+  if (kv_head_begin < 0 || kv_head_end <= kv_head_begin || kv_head_end > shape->num_kv_heads)
+    return WAITS_ERR_ARG;
+  if (!Q || !K || !V) return WAITS_ERR_ARG;
+  // the heads [begin, end) of the layer as a layer of their own: the same
+  // token rows (rows keep the layer's head count), shifted base pointers
+  const int G = shape->num_q_heads / shape->num_kv_heads, d = shape->head_dim;
+  waits_shape sub = *shape;
+  sub.num_kv_heads = kv_head_end - kv_head_begin;
+  sub.num_q_heads = sub.num_kv_heads * G;
+  const uint16_t* Qs = static_cast<const uint16_t*>(Q) + (size_t)kv_head_begin * G * d;
+  const uint16_t* Ks = static_cast<const uint16_t*>(K) + (size_t)kv_head_begin * d;
+  const uint16_t* Vs = static_cast<const uint16_t*>(V) + (size_t)kv_head_begin * d;
+  st = check_score_args(&sub, Qs, Ks, a, b, scores);
+  if (st == WAITS_OK) st = check_select_args(scores, R, B, idx, kept_len);
+  if (st == WAITS_OK) st = check_compact_args(Ks, Vs, idx, kept_len, B, K_out, V_out);
+  if (st == WAITS_OK) st = check_ws(&sub, workspace, workspace_bytes);
+  if (st != WAITS_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = enqueue_score(&sub, Qs, Ks, a, b, scores, workspace, s, nullptr, nullptr, nullptr,
+                     shape->num_q_heads, shape->num_kv_heads);
+  if (st != WAITS_OK) return st;
+  const cudaError_t err = launch_select(
+      scores, sub.cu_seqlens, sub.nseq, sub.total_tokens, sub.num_kv_heads, R, B, idx, kept_len,
+      status_word(workspace, workspace_bytes), s, Ks, Vs, d, static_cast<uint16_t*>(K_out),
+      static_cast<uint16_t*>(V_out), shape->num_kv_heads);
+  if (err != cudaSuccess) return cuda_fail("select-compact launch", err);
+  return WAITS_OK;
+}
+
 waits_status waits_select_compact(const waits_shape* shape, const float* scores,
                                   const void* K, const void* V, int32_t R, int32_t B,
                                   int32_t* idx, int32_t* kept_len, void* K_out, void* V_out,
@@ -476,6 +516,46 @@ waits_status waits_compress_host(const waits_shape* shape, const int32_t* cu_hos
   if (!ok) return WAITS_ERR_CUDA;
   if (h2d_bytes) *h2d_bytes = up;
   if (d2h_bytes) *d2h_bytes = down;
+  return WAITS_OK;
+}
+
+waits_status decode_dims_ok(int32_t nseq, int32_t Hq, int32_t Hkv, int32_t d, int32_t C) {
+  if (nseq < 1 || Hq < 1 || Hkv < 1 || C < 1 || Hq % Hkv) return WAITS_ERR_SHAPE;
+  if (d != 64 && d != 128) return WAITS_ERR_UNSUPPORTED;
+  if (Hq / Hkv > decode_max_group()) return WAITS_ERR_UNSUPPORTED;
+  if ((int64_t)nseq * Hkv > 65535LL * 65535LL || Hq > 65535 || nseq > 65535)
+    return WAITS_ERR_SHAPE;
+  return WAITS_OK;
+}
+
+waits_status waits_decode_workspace_size(int32_t nseq, int32_t num_q_heads, int32_t head_dim,
+                                         int32_t capacity, size_t* bytes) {
+  if (!bytes) return WAITS_ERR_ARG;
+  if (nseq < 1 || num_q_heads < 1 || capacity < 1) return WAITS_ERR_SHAPE;
+  if (head_dim != 64 && head_dim != 128) return WAITS_ERR_UNSUPPORTED;
+  *bytes = decode_workspace_bytes(nseq, num_q_heads, head_dim, capacity);
+  return WAITS_OK;
+}
+
+waits_status waits_decode_attention(int32_t nseq, int32_t num_q_heads, int32_t num_kv_heads,
+                                    int32_t head_dim, int32_t capacity, const void* q,
+                                    const void* K_cache, const void* V_cache,
+                                    const int32_t* cache_len, float* out, float* lse,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  waits_status st = decode_dims_ok(nseq, num_q_heads, num_kv_heads, head_dim, capacity);
+  if (st != WAITS_OK) return st;
+  if (!q || !K_cache || !V_cache || !cache_len || !out) return WAITS_ERR_ARG;
+  if (!aligned(q, 16) || !aligned(K_cache, 16) || !aligned(V_cache, 16) || !aligned(out, 4) ||
+      !aligned(cache_len, 4) || (lse && !aligned(lse, 4)))
+    return WAITS_ERR_ARG;
+  if (!workspace || !aligned(workspace, 16) ||
+      workspace_bytes < decode_workspace_bytes(nseq, num_q_heads, head_dim, capacity))
+    return WAITS_ERR_WORKSPACE;
+  const cudaError_t err = launch_decode(
+      nseq, num_q_heads, num_kv_heads, head_dim, capacity, static_cast<const uint16_t*>(q),
+      static_cast<const uint16_t*>(K_cache), static_cast<const uint16_t*>(V_cache), cache_len,
+      out, lse, static_cast<float*>(workspace), static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail("decode launch", err);
   return WAITS_OK;
 }
 

@@ -225,9 +225,10 @@ struct PlanArgs {
 };
 
 struct PassArgs {
-  const uint16_t* Q;   // bf16 bits [T, Hq, d]
-  const uint16_t* K;   // bf16 bits [T, Hkv, d]
+  const uint16_t* Q;   // bf16 bits [T, Hq, d] (rows of q_row_heads heads)
+  const uint16_t* K;   // bf16 bits [T, Hkv, d] (rows of kv_row_heads heads)
   int T, Hq, Hkv, G, tokq, d;
+  int q_row_heads, kv_row_heads;   // heads per token row in memory (>= Hq, Hkv)
   float a;
   int b;
   float scale2;        // log2(e) / sqrt(d)
@@ -323,10 +324,16 @@ cudaError_t launch_select(const float* scores, const int32_t* cu, int nseq, int 
                           int Hkv, int R, int B, int32_t* idx, int32_t* kept_len,
                           uint32_t* status, cudaStream_t s, const uint16_t* K = nullptr,
                           const uint16_t* V = nullptr, int d = 0, uint16_t* Ko = nullptr,
-                          uint16_t* Vo = nullptr);
+                          uint16_t* Vo = nullptr, int kv_row_heads = 0);
 cudaError_t launch_compact(const uint16_t* K, const uint16_t* V, const int32_t* cu,
                            const int32_t* idx, const int32_t* kept_len, int nseq,
                            int Hkv, int d, int B, uint16_t* Ko, uint16_t* Vo,
-                           uint32_t* status, cudaStream_t s);
+                           uint32_t* status, cudaStream_t s, int kv_row_heads = 0);
+// Decode attention over the compacted cache (decode.cu).
+size_t decode_workspace_bytes(int64_t nseq, int64_t Hq, int64_t d, int64_t C);
+int decode_max_group();
+cudaError_t launch_decode(int nseq, int Hq, int Hkv, int d, int C, const uint16_t* q,
+                          const uint16_t* Kc, const uint16_t* Vc, const int32_t* len, float* out,
+                          float* lse, float* part, cudaStream_t st);
 
 }  // namespace waits

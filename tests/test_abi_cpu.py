@@ -188,3 +188,23 @@ def test_score_kernel_count(lib):
     assert _kernels(lib, llama8b, -1.0, 16)[0] == 1
     assert _kernels(lib, llama8b, 1.0, -1)[0] == 1
     assert lib.waits_score_kernels(ctypes.byref(llama8b), 1.0, 16, None) == 1
+
+
+def test_decode_argument_errors(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.waits_decode_workspace_size(1, 32, 128, 2048, None) == 1
+    assert lib.waits_decode_workspace_size(1, 32, 96, 2048, ctypes.byref(n)) == 3
+    assert lib.waits_decode_workspace_size(1, 32, 128, 2048, ctypes.byref(n)) == 0
+    assert n.value == 32 * 8 * 130 * 4
+    F = 0x100000
+
+    def call(nseq=1, Hq=32, Hkv=8, d=128, C=2048, q=F, k=F, v=F, ln=F, out=F, ws=F, wsb=10**7):
+        return lib.waits_decode_attention(nseq, Hq, Hkv, d, C, q, k, v, ln, out, None, ws, wsb,
+                                          None)
+
+    assert call(Hq=30) == 2                 # Hq not a multiple of Hkv
+    assert call(d=80) == 3                  # head dim
+    assert call(Hq=32, Hkv=1) == 3          # G > 16
+    assert call(q=0) == 1 and call(out=0) == 1
+    assert call(q=F + 8) == 1               # 16-byte alignment
+    assert call(wsb=16) == 4                # workspace too small
