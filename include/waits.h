@@ -389,10 +389,12 @@ waits_status waits_decode_attention(int32_t nseq, int32_t num_q_heads, int32_t n
  * Testing aid, no counterpart on the WAITS pages: y[i] = the scorer's
  * FMA-pipe 2^x of x[i] (the exponential that part of the scorer's epilogue
  * runs instead of the MUFU ex2: a round-to-nearest split x = n + f, a cubic
- * in f with relative error 1.013e-4 (1.02e-4 with fp32 rounding), 2^n
- * added to the exponent; x is first clamped to [-125, 127]).  x and y are
- * DEVICE fp32 arrays of n elements.  Errors: ARG (null pointer, n < 0),
- * CUDA.
+ * in f with relative error 1.013e-4 (1.02e-4 with fp32 rounding), 2^n built
+ * from the bits of the rounding sum).  x is first raised to at least -127,
+ * so x <= -126.5 gives +0; defined for x <= 127 (the epilogue's arguments
+ * never exceed 0 beyond rounding); exact powers of two at integers in
+ * [-126, 127].  x and y are DEVICE fp32 arrays of n elements.  Errors: ARG
+ * (null pointer, n < 0), CUDA.
  */
 waits_status waits_test_exp2_poly(const float* x, float* y, int64_t n, void* stream);
 

@@ -288,15 +288,14 @@ __device__ void s_epilogue_p1(const PassArgs& p, SB sm, const SeqInfo* seqs, con
       if (ok && !mbar_wait(sm.bar(L::tfull, w), ph, abort, p.status, p.wait_ns)) ok = false;
       if (!ok) continue;
       tc_fence_after();
-      Cols v;
-      v.load_wait(lane_addr);
-      if (n == 1) release_acc(sm.bar(L::tempty, w), lane);
-      int nv = row_tok >= 0 ? row_tok - o * kTile + 1 : 0;
-      p1_pair(v, nv > kTile ? kTile : nv, p.scale2, m, l);
-      if (n == 2) {
-        v.load_wait(lane_addr + kTile);
-        release_acc(sm.bar(L::tempty, w), lane);
-        nv = row_tok >= 0 ? row_tok - (o + 1) * kTile + 1 : 0;
+      // the accumulator's halves in one loop: one copy of the unrolled
+      // arithmetic in the instruction stream
+#pragma unroll 1
+      for (int h = 0; h < n; ++h) {
+        Cols v;
+        v.load_wait(lane_addr + (uint32_t)(h * kTile));
+        if (h == n - 1) release_acc(sm.bar(L::tempty, w), lane);
+        const int nv = row_tok >= 0 ? row_tok - (o + h) * kTile + 1 : 0;
         p1_pair(v, nv > kTile ? kTile : nv, p.scale2, m, l);
       }
     }
@@ -352,16 +351,17 @@ __device__ void s_epilogue_p2(const PassArgs& p, SB sm, const SeqInfo* seqs, con
         if (ok && !mbar_wait(sm.bar(L::tfull, w), ph, abort, p.status, p.wait_ns)) ok = false;
         if (ok) {
           tc_fence_after();
-          Cols v;
-          v.load_wait(lane_addr);
-          if (!ex1) release_acc(sm.bar(L::tempty, w), lane);
-          if (live0) col += p2_pair(v, key > f0 ? min((key - f0) * p.G, kTile) : 0, nc0,
-                                    p.scale2, bias0);
-          if (ex1) {
-            v.load_wait(lane_addr + kTile);
-            release_acc(sm.bar(L::tempty, w), lane);
-            if (live1) col += p2_pair(v, key > f1 ? min((key - f1) * p.G, kTile) : 0, nc1,
-                                      p.scale2, bias1);
+          // both Q tiles in one loop: one copy of the unrolled arithmetic
+          const int nh = ex1 ? 2 : 1;
+#pragma unroll 1
+          for (int h = 0; h < nh; ++h) {
+            Cols v;
+            v.load_wait(lane_addr + (uint32_t)(h * kTile));
+            if (h == nh - 1) release_acc(sm.bar(L::tempty, w), lane);
+            const bool live = h == 0 ? live0 : live1;
+            const int f = h == 0 ? f0 : f1;
+            if (live) col += p2_pair(v, key > f ? min((key - f) * p.G, kTile) : 0,
+                                     h == 0 ? nc0 : nc1, p.scale2, h == 0 ? bias0 : bias1);
           }
         }
       }

@@ -519,15 +519,17 @@ cudaError_t launch_d(const PassArgs& a, const HostPlan& hp, int grid, cudaStream
 }  // namespace
 
 // The scorer's FMA-pipe 2^x on n values (a testing aid: the same function
-// the epilogue runs, so its error can be measured against exact powers).
+// the epilogue runs, added to zero, so its error can be measured against
+// exact powers).
 __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
   const int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  const float2 zero = make_float2(0.f, 0.f);
   if (i + 1 < n) {
-    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    const float2 r = exp2_poly_acc(make_float2(x[i], x[i + 1]), zero);
     y[i] = r.x;
     y[i + 1] = r.y;
   } else if (i < n) {
-    y[i] = exp2_poly2(make_float2(x[i], 0.f)).x;
+    y[i] = exp2_poly_acc(make_float2(x[i], 0.f), zero).x;
   }
 }
 

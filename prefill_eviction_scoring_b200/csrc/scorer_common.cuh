@@ -67,35 +67,49 @@ __device__ inline float hsum8(const float2 (&a)[4]) {
 
 // Column pairs whose exponential runs on the FMA pipe instead of the MUFU
 // (which does 16 ex2 per clock per SM and bounds the unmasked passes): bit
-// (pair index mod 8) of this mask.  Two in eight measured best with the
-// 256-column accumulators (one in eight 3 % slower, three in eight 4 %).
-constexpr uint32_t kPolyPairs = 0x88u;
+// (pair index mod 8) of this mask.  Three in eight measured best with the
+// shift-add exponential below (an epilogue-only loop over TMEM tiles: pass 1
+// 885 clocks per 128x128 tile against 1096 with the MUFU alone, pass 2 865;
+// two in eight 995 / 905, four in eight 951 / 906).
+constexpr uint32_t kPolyPairs = 0x92u;
 __device__ constexpr bool poly_col(int c) { return (kPolyPairs >> ((c >> 1) & 7)) & 1u; }
 
-// 2^x for a pair of fp32 values on the FMA/ALU pipes (Cody-Waite split plus
-// a polynomial): x = n + f with n = rint(x) and f in [-1/2, 1/2];
+// acc + 2^x for a pair of fp32 values on the FMA/ALU pipes (Cody-Waite split
+// plus a polynomial): x = n + f with n = rint(x) and f in [-1/2, 1/2];
 // 2^f ~ 1 + f (c1 + f (c2 + f c3)), the relative-error minimax cubic with the
 // constant term held at 1 (max relative error 1.013e-4; fitted by linear
-// programming on a dense grid), so integer x gives exact powers of two; 2^n
-// is added to the exponent bits.  x is clamped to [-125, 127] so the result
-// stays a normal fp32 number.
-__device__ inline float2 exp2_poly2(float2 x) {
-  constexpr float kMagic = 12582912.0f;              // 1.5 * 2^23: rint via fadd
+// programming on a dense grid), so integer x gives exact powers of two.
+// rint comes from adding 1.5 * 2^23 + 127: the sum's low mantissa bits are
+// then n + 127, so shifting its bit pattern left by 23 leaves exactly the
+// fp32 pattern of 2^n (the magic's own bits above bit 8 shift out); the
+// product with the cubic is fused into the running sum.  x is raised to at
+// least -127, whose pattern is +0, so x <= -126.5 adds nothing (as the MUFU's
+// flush to zero does below 2^-126).  Valid for x <= 127: every argument the
+// epilogue forms is at most 0 up to rounding (a logit minus the row maximum,
+// or a bias that includes the row's log-sum-exp).
+__device__ inline float2 exp2_poly_acc(float2 x, float2 acc) {
+  constexpr float kMagic = 12582912.0f + 127.0f;     // exact in fp32
   constexpr float c1 = 0.69328290f, c2 = 0.24221097f, c3 = 0.05500906f;
-  x = f2(fminf(fmaxf(x.x, -125.f), 127.f), fminf(fmaxf(x.y, -125.f), 127.f));
+  x = f2(fmaxf(x.x, -127.f), fmaxf(x.y, -127.f));
   const float2 t = __fadd2_rn(x, f2(kMagic, kMagic));
   const float2 n = __fadd2_rn(t, f2(-kMagic, -kMagic));
   const float2 fr = __ffma2_rn(n, f2(-1.f, -1.f), x);
   float2 q = __ffma2_rn(f2(c3, c3), fr, f2(c2, c2));
   q = __ffma2_rn(q, fr, f2(c1, c1));
   q = __ffma2_rn(q, fr, f2(1.f, 1.f));
-  // the magic's low 9 bits are zero, so (bits(t) << 23) == n << 23
-  const int ex = __float_as_int(t.x) << 23, ey = __float_as_int(t.y) << 23;
-  return f2(__int_as_float(__float_as_int(q.x) + ex), __int_as_float(__float_as_int(q.y) + ey));
+  const float2 p = f2(__int_as_float(__float_as_int(t.x) << 23),
+                      __int_as_float(__float_as_int(t.y) << 23));
+  return __ffma2_rn(q, p, acc);
 }
 
-// sum_c 2^(v_c * sc + off) over all 128 columns, packed fp32x2 arithmetic;
-// the column pairs picked by kPolyPairs use the polynomial, the rest the MUFU.
+// acc + 2^x for a column pair: the polynomial for the pairs of kPolyPairs,
+// else the MUFU.
+__device__ inline float2 exp2_add(int c, float2 x, float2 acc) {
+  return poly_col(c) ? exp2_poly_acc(x, acc)
+                     : __fadd2_rn(acc, f2(ex2_approx(x.x), ex2_approx(x.y)));
+}
+
+// sum_c 2^(v_c * sc + off) over all 128 columns, packed fp32x2 arithmetic.
 __device__ inline float exp_sum_full(const Cols& v, float sc, float off) {
   const float2 sc2 = f2(sc, sc), off2 = f2(off, off);
   float2 a[4];
@@ -104,8 +118,7 @@ __device__ inline float exp_sum_full(const Cols& v, float sc, float off) {
 #pragma unroll
   for (int c = 0; c < kTile; c += 2) {
     const float2 x = __ffma2_rn(f2(u2f(v.r[c]), u2f(v.r[c + 1])), sc2, off2);
-    const float2 e = poly_col(c) ? exp2_poly2(x) : f2(ex2_approx(x.x), ex2_approx(x.y));
-    a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], e);
+    a[(c >> 1) & 3] = exp2_add(c, x, a[(c >> 1) & 3]);
   }
   return hsum8(a);
 }
@@ -131,15 +144,22 @@ __device__ inline float exp_sum_masked(const Cols& v, int nv, float sc, float of
   return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
-// Largest raw value of the whole tile (8 independent chains).
+// max(a, b, c) in one instruction (the three-input form sm_100 has).
+__device__ inline float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Largest raw value of the whole tile (8 independent chains of three-input
+// maxima).
 __device__ inline float tile_max_raw(const Cols& v) {
   float mx[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) mx[k] = u2f(v.r[k]);
 #pragma unroll
-  for (int c = 8; c < kTile; ++c) mx[c & 7] = fmaxf(mx[c & 7], u2f(v.r[c]));
-  return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+  for (int c = 8; c < kTile; c += 2) mx[(c >> 1) & 7] = fmax3(mx[(c >> 1) & 7], u2f(v.r[c]), u2f(v.r[c + 1]));
+  return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 }
 
 // Pass 1, one 128-key tile of this thread's row (keys c < nv are causal):
@@ -183,11 +203,8 @@ __device__ inline float p2_pair(const Cols& v, int c_lo, int ncols, float sc, co
           const float4 b = b4[c / 4];
           const float2 x0 = __ffma2_rn(f2(u2f(v.r[c]), u2f(v.r[c + 1])), sc2, f2(b.x, b.y));
           const float2 x1 = __ffma2_rn(f2(u2f(v.r[c + 2]), u2f(v.r[c + 3])), sc2, f2(b.z, b.w));
-          const float2 e0 = poly_col(c) ? exp2_poly2(x0) : f2(ex2_approx(x0.x), ex2_approx(x0.y));
-          const float2 e1 =
-              poly_col(c + 2) ? exp2_poly2(x1) : f2(ex2_approx(x1.x), ex2_approx(x1.y));
-          a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], e0);
-          a[((c >> 1) + 1) & 3] = __fadd2_rn(a[((c >> 1) + 1) & 3], e1);
+          a[(c >> 1) & 3] = exp2_add(c, x0, a[(c >> 1) & 3]);
+          a[((c >> 1) + 1) & 3] = exp2_add(c + 2, x1, a[((c >> 1) + 1) & 3]);
         }
       }
     }

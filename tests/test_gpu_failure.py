@@ -5,9 +5,10 @@
   out after a short limit; the call must end with WAITS_DEV_TIMEOUT in the
   status word, without a fault or a hang, and the next normal call on the
   same context must be clean and correct.
-* exp2_poly2, the 2^x that part of the epilogue computes on the FMA pipe:
-  relative error at most 1.02e-4 against exact powers of two over the clamp
-  range [-125, 127], exact at integers, clamped outside.
+* exp2_poly_acc, the 2^x that part of the epilogue computes on the FMA pipe:
+  relative error at most 1.02e-4 against exact powers of two over
+  [-125, 127], exact at integers, zero at and below -127 (its clamp), and
+  within the bound down to -126.5 where the result becomes subnormal.
 """
 
 import ctypes
@@ -84,10 +85,16 @@ def test_exp2_poly_relative_error_bound():
 
 @pytest.mark.gpu
 def test_exp2_poly_exact_at_integers_and_clamped():
-    n = np.arange(-125, 128, dtype=np.float32)
+    n = np.arange(-126, 128, dtype=np.float32)
     y = _exp2_poly(torch.from_numpy(n).cuda()).cpu().numpy()
     np.testing.assert_array_equal(y, np.exp2(n.astype(np.float64)).astype(np.float32))
-    far = np.array([-1e30, -1000.0, -126.0, -125.5, 127.5, 128.0, 500.0, 1e30], dtype=np.float32)
+    # raised to -127, whose 2^n pattern is +0: nothing below, like a flush to zero
+    far = np.array([-np.inf, -1e30, -1000.0, -127.0, -126.75, -126.5], dtype=np.float32)
     y = _exp2_poly(torch.from_numpy(far).cuda()).cpu().numpy()
-    lo, hi = np.float32(2.0 ** -125), np.float32(2.0 ** 127)
-    np.testing.assert_array_equal(y, [lo, lo, lo, lo, hi, hi, hi, hi])
+    np.testing.assert_array_equal(y, np.zeros(len(far), dtype=np.float32))
+    assert not np.signbit(y).any()
+    # n = -126 with f in (-1/2, 1/2]: 2^-126 times the cubic, subnormal below 2^-126
+    x = np.linspace(-126.49, -125.51, 99).astype(np.float32)
+    y = _exp2_poly(torch.from_numpy(x).cuda()).cpu().numpy().astype(np.float64)
+    ref = np.exp2(x.astype(np.float64))
+    assert (np.abs(y - ref) / ref).max() <= 1.02e-4
