@@ -49,10 +49,12 @@ EVENT_EVERY = 8         # stack workloads: CUDA events around every 8th layer's 
 MUFU_EX2_PER_CLK_PER_SM = 16   # sm_100: 4 SFU lanes per SM sub-partition x 4
 L2_BYTES = 126 << 20
 # DRAM bytes (read + write) of one waits_score call on one 8B-shaped layer
-# (N = 32768, a = 1, b = 16) from the committed ncu capture of the scorer
-# (both passes).  Valid only for the scorer source it was taken on.
-PROFILED_SCORER = {"sha256_prefix": "c4dc12a0abdeda18", "dram_bytes": 68_140_032 + 1_554_176 +
-                   68_432_640 + 1_249_536}
+# (N = 32768, a = 1, b = 16) from the committed ncu capture of the sparse
+# scorer (both passes).  Valid only for the scorer sources it was taken on
+# (sha256 of score_sparse.cu followed by scorer_common.cuh).
+PROFILED_SCORER = {"sha256_prefix": "b2e4d786d37e919a",
+                   "dram_bytes": 68_208_640 + 1_739_264 + 68_376_320 + 1_047_040}
+PROFILED_SOURCES = ("score_sparse.cu", "scorer_common.cuh")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -238,16 +240,23 @@ def rooflines(lens, Hq, Hkv, d, a, b, B, t_score_ms, t_sc_ms, layer_ms, pk, sm_c
     return head, other
 
 
+def scorer_source_hash() -> str:
+    """sha256 of the sparse scorer's sources, in PROFILED_SOURCES order."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in PROFILED_SOURCES:
+        with open(os.path.join(ROOT, "prefill_eviction_scoring_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def profiled_traffic(case: Case):
     """ncu DRAM bytes of the scorer for the headline layer, or None when the
-    case differs or score_tc.cu has changed since the capture."""
-    import hashlib
+    case differs or the scorer's sources have changed since the capture."""
     if (case.config, case.a, case.b) != ("llama8b", 1.0, 16) or case.name != "llama8b":
         return None
-    src = os.path.join(ROOT, "prefill_eviction_scoring_b200", "csrc", "score_tc.cu")
-    with open(src, "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()
-    return PROFILED_SCORER["dram_bytes"] if h.startswith(PROFILED_SCORER["sha256_prefix"]) else None
+    ok = scorer_source_hash().startswith(PROFILED_SCORER["sha256_prefix"])
+    return PROFILED_SCORER["dram_bytes"] if ok else None
 
 
 def oracle_active_logits(N, a, b):
