@@ -745,6 +745,13 @@ def run_case(args, D, lib, case: Case, headline: bool):
                    f"buffers; the kept V rows are read in place over the bus)"
                    + (f", alternating over {NS} streams" if NS > 1 else ""),
            "ms_per_step": round(e2e_ms, 3)}
+    # the host link carries every input and output byte of the step: its rate
+    # says how much of the step the transfers alone account for
+    e2e["host_link_gbs"] = round((e2e["h2d_bytes_per_step"] + e2e["d2h_bytes_per_step"])
+                                 / (e2e_ms / 1e3) / 1e9, 1)
+    e2e["note"] = ("bound by the host link, not the kernels: each step moves "
+                   f"{(e2e['h2d_bytes_per_step'] + e2e['d2h_bytes_per_step']) / 1e6:.0f} MB "
+                   f"at {e2e['host_link_gbs']} GB/s; the device-resident line is `value`")
 
     cpu = None
     if D.rank == 0 and D.world == 1 and not args.no_cpu_baseline:
