@@ -405,8 +405,9 @@ waits_status waits_test_exp2_poly(const float* x, float* y, int64_t n, void* str
  * makes the scorer's MMA warp issue nothing, so the waits for its
  * accumulators run out: the call ends early, with WAITS_DEV_TIMEOUT set and
  * the scores unspecified, and leaves the context usable.  WAITS_SCORER=tc
- * makes small plans run the general scorer kernel instead of the one for
- * sparse weights (the scores are bit-identical either way).
+ * makes both passes of every plan run the general scorer kernel (by
+ * default the kernel with 256-column accumulators runs pass 1 of every plan
+ * and pass 2 of the small ones; the scores are bit-identical either way).
  */
 
 #ifdef __cplusplus

@@ -442,24 +442,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_wait();
     pdl_allow_next();
   }
-  LocalPlan* lp = sm.at<LocalPlan>(L::lp);
-  {
-    PassArgs q = pa;
-    plan_prologue(q, pa, hp, lp, p1, warp);
-  }
-  const Entry* E = p1 ? lp->e1 : lp->e2;
+  // the plan: this CTA's own (local plans) or the planner kernel's, in the
+  // workspace (pass 1 of a large plan, whose pass 2 the general kernel runs)
+  PassArgs q = pa;
+  plan_prologue(q, pa, hp, sm.at<LocalPlan>(L::lp), p1, warp);
+  const Entry* E = p1 ? q.e1 : q.e2;
+  const SeqInfo* seqs = q.seqs;
 
   UnitIter it;
-  const PlanHeader& H = lp->hdr;
+  const PlanHeader& H = *q.hdr;
   const bool have = it.init(E, p1 ? H.n_e1 : H.n_e2, p1 ? H.s1 : H.s2, p1 ? H.p1 : H.p2,
                             blockIdx.x, (p1 ? H.aligned1 : H.aligned2) != 0);
   if (warp >= kProducerWarp) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
     if (have && warp == kProducerWarp) {
-      if (lane == 0) s_producer<D, PASS>(&tmQ, &tmK, pa, sm, lp->seqs, E, it);
+      if (lane == 0) s_producer<D, PASS>(&tmQ, &tmK, pa, sm, seqs, E, it);
       __syncwarp();
     } else if (have && warp == kMmaWarp) {
-      if (lane == 0) s_mma<D, PASS>(pa, sm, lp->seqs, E, it, tmem);
+      if (lane == 0) s_mma<D, PASS>(pa, sm, seqs, E, it, tmem);
       __syncwarp();
     }
   } else {
@@ -469,8 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       pdl_allow_next();
     }
     if (have) {
-      if (p1) s_epilogue_p1<D>(pa, sm, lp->seqs, E, it, tmem);
-      else s_epilogue_p2<D>(pa, sm, lp->seqs, lp->e1, E, it, tmem);
+      if (p1) s_epilogue_p1<D>(pa, sm, seqs, E, it, tmem);
+      else s_epilogue_p2<D>(pa, sm, seqs, q.e1, E, it, tmem);
     }
   }
   tc_fence_before();
@@ -490,7 +490,8 @@ static_assert(sizeof(HostPlan) + 2 * sizeof(CUtensorMap) + sizeof(PassArgs) + 64
               "scorer parameters must stay within 4 KB");
 
 template <int D>
-cudaError_t launch_sparse_d(const PassArgs& a, const HostPlan& hp, int grid, cudaStream_t st) {
+cudaError_t launch_sparse_d(const PassArgs& a, const HostPlan& hp, int grid, cudaStream_t st,
+                            bool pass2 = true) {
   CUtensorMap mq, mk;
   if (!make_map(&mq, a.Q, a.T, a.Hq, a.q_row_heads, D, a.G, a.tokq) ||
       !make_map(&mk, a.K, a.T, a.Hkv, a.kv_row_heads, D, 1, kTile))
@@ -507,6 +508,7 @@ cudaError_t launch_sparse_d(const PassArgs& a, const HostPlan& hp, int grid, cud
   if (!a.lse && (err = launch_pdl(score_sparse_kernel<D, 1>, dim3(grid), dim3(kThreads), smem1,
                                   st, mq, mk, a, hp)) != cudaSuccess)
     return err;
+  if (!pass2) return cudaSuccess;
   return launch_pdl(score_sparse_kernel<D, 2>, dim3(grid), dim3(kThreads), smem2, st, mq, mk, a,
                     hp);
 }
@@ -518,6 +520,12 @@ cudaError_t launch_sparse_passes(const PassArgs& a, const HostPlan* hp, int grid
   static const HostPlan kNone{};
   const HostPlan& h = hp ? *hp : kNone;
   return a.d == 64 ? launch_sparse_d<64>(a, h, grid, s) : launch_sparse_d<128>(a, h, grid, s);
+}
+
+cudaError_t launch_sparse_pass1(const PassArgs& a, int grid, cudaStream_t s) {
+  static const HostPlan kNone{};
+  return a.d == 64 ? launch_sparse_d<64>(a, kNone, grid, s, false)
+                   : launch_sparse_d<128>(a, kNone, grid, s, false);
 }
 
 }  // namespace waits

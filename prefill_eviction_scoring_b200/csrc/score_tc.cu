@@ -484,7 +484,8 @@ static_assert(sizeof(HostPlan) + 2 * sizeof(CUtensorMap) + sizeof(PassArgs) + 64
               "scorer parameters must stay within 4 KB");
 
 template <int D>
-cudaError_t launch_d(const PassArgs& a, const HostPlan& hp, int grid, cudaStream_t st) {
+cudaError_t launch_d(const PassArgs& a, const HostPlan& hp, int grid, cudaStream_t st,
+                     bool pass1 = true) {
   CUtensorMap mq, mk;
   if (!make_map(&mq, a.Q, a.T, a.Hq, a.q_row_heads, D, a.G, a.tokq) ||
       !make_map(&mk, a.K, a.T, a.Hkv, a.kv_row_heads, D, 1, kTile))
@@ -498,8 +499,9 @@ cudaError_t launch_d(const PassArgs& a, const HostPlan& hp, int grid, cudaStream
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) !=
           cudaSuccess)
     return err;
-  if (!a.lse && (err = launch_pdl(score_tc_kernel<D, 1>, dim3(grid), dim3(kThreads), smem1, st,
-                                  mq, mk, a, hp)) != cudaSuccess) {
+  if (pass1 && !a.lse &&
+      (err = launch_pdl(score_tc_kernel<D, 1>, dim3(grid), dim3(kThreads), smem1, st, mq, mk, a,
+                        hp)) != cudaSuccess) {
     cudaFuncAttributes fa{};
     cudaFuncGetAttributes(&fa, score_tc_kernel<D, 1>);
     int dev = 0, optin = 0, regs = 0;
@@ -545,6 +547,12 @@ cudaError_t launch_score_passes(const PassArgs& a, const HostPlan* hp, int grid,
   static const HostPlan kNone{};
   const HostPlan& h = hp ? *hp : kNone;
   return a.d == 64 ? launch_d<64>(a, h, grid, s) : launch_d<128>(a, h, grid, s);
+}
+
+cudaError_t launch_score_pass2(const PassArgs& a, int grid, cudaStream_t s) {
+  static const HostPlan kNone{};
+  return a.d == 64 ? launch_d<64>(a, kNone, grid, s, false)
+                   : launch_d<128>(a, kNone, grid, s, false);
 }
 
 }  // namespace waits

@@ -197,10 +197,17 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
                         host_plan_single(p.T, p.max_seqlen, p.Hkv, p.tokq, a, b, grid, &hp)
                     ? 1
                     : 0;
-  // local plans hold only P2Q entries in pass 2: the 256-column kernel
-  err = local && !force_tc_scorer()
-            ? launch_sparse_passes(p, p.host_plan ? &hp : nullptr, grid, st)
-            : launch_score_passes(p, p.host_plan ? &hp : nullptr, grid, st);
+  // local plans hold only P2Q entries in pass 2: the 256-column kernel for
+  // both passes; the planner kernel's plans: its pass 1, and the general
+  // kernel's pass 2 (which also handles stationary K tiles)
+  if (force_tc_scorer())
+    err = launch_score_passes(p, p.host_plan ? &hp : nullptr, grid, st);
+  else if (local)
+    err = launch_sparse_passes(p, p.host_plan ? &hp : nullptr, grid, st);
+  else if (lse)
+    err = launch_score_passes(p, nullptr, grid, st);   // pass 2 only
+  else if ((err = launch_sparse_pass1(p, grid, st)) == cudaSuccess)
+    err = launch_score_pass2(p, grid, st);
   if (err != cudaSuccess) return cuda_fail("scorer launch", err);
   return WAITS_OK;
 }

@@ -317,6 +317,10 @@ cudaError_t launch_score_passes(const PassArgs& a, const HostPlan* hp, int grid,
 // The same two passes for a local plan (every entry of pass 2 in mode P2Q):
 // 256-column accumulators, bit-identical scores.
 cudaError_t launch_sparse_passes(const PassArgs& a, const HostPlan* hp, int grid, cudaStream_t s);
+// Large plans (the planner kernel's, in the workspace): pass 1 by the
+// 256-column kernel (bit-identical row partials), pass 2 by score_tc.cu's.
+cudaError_t launch_sparse_pass1(const PassArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_score_pass2(const PassArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
 // K == nullptr: selection only; else also the compaction of K and V into
 // Ko, Vo (the rows of the kept positions, zeros past kept_len).
