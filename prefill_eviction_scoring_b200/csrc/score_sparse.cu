@@ -438,6 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Pass 1 waits for whatever wrote Q, K and cu_seqlens before anything,
   // then lets pass 2 launch; pass 2's copy and MMA warps start at once, only
   // its epilogue waits (below) for pass 1's row partials.
+  stage_host_plan(pa, hp, sm.at<LocalPlan>(L::lp));
   if (p1 || pa.lse) {
     pdl_wait();
     pdl_allow_next();

@@ -443,6 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // then lets pass 2 launch: from then on the plan, Q and K are complete, so
   // pass 2's copy and MMA warps start on them at once; only its epilogue
   // waits (below) for pass 1's row biases.
+  stage_host_plan(pa, hp, s.lp);
   if (p1 || pa.lse) {
     pdl_wait();
     pdl_allow_next();

@@ -336,10 +336,29 @@ __device__ inline void qrow_bias(const PassArgs& p, const SeqInfo& si, int g, co
   qrow_bias<NR>(p, p.e1, si, g, j, r, out);
 }
 
+// The host's one-sequence plan into this CTA's shared memory.  It is a
+// kernel parameter, so this runs before the wait for the previous kernel;
+// plan_prologue then only checks cu_seqlens and writes the header.
+__device__ inline void stage_host_plan(const PassArgs& pa, const HostPlan& hp, LocalPlan* lp) {
+  if (!pa.local_plan || !pa.host_plan) return;
+  constexpr int kVecs = (int)(sizeof(Entry) / sizeof(uint4));
+  const int n1 = hp.hdr.n_e1, n2 = hp.hdr.n_e2;
+  const uint4* h1 = reinterpret_cast<const uint4*>(hp.e1);
+  const uint4* h2 = reinterpret_cast<const uint4*>(hp.e2);
+  uint4* d1 = reinterpret_cast<uint4*>(lp->e1);
+  uint4* d2 = reinterpret_cast<uint4*>(lp->e2);
+  for (int i = threadIdx.x; i < (n1 + n2) * kVecs; i += blockDim.x) {
+    if (i < n1 * kVecs) d1[i] = h1[i];
+    else d2[i - n1 * kVecs] = h2[i - n1 * kVecs];
+  }
+  if (threadIdx.x == 0) lp->seqs[0] = hp.seq;
+}
+
 // Every CTA's share of the plan: with a local plan each CTA builds it in
-// shared memory (or copies the host's one-sequence plan) and points `p` at
-// it; pass 1 also resets the call's status word and zeroes the scores of
-// sequences without an active row.  Called by all threads of the CTA.
+// shared memory (or takes the host's one-sequence plan, staged before the
+// wait) and points `p` at it; pass 1 also resets the call's status word and
+// zeroes the scores of sequences without an active row.  Called by all
+// threads of the CTA.
 __device__ inline void plan_prologue(PassArgs& p, const PassArgs& pa, const HostPlan& hp,
                                      LocalPlan* lp, bool p1, int warp) {
   if (p.local_plan) {
@@ -347,19 +366,10 @@ __device__ inline void plan_prologue(PassArgs& p, const PassArgs& pa, const Host
     // above, and pass 2 starts only after pass 1 has), or copies the plan
     // the host built for the batch {0, T} once cu_seqlens reads so
     if (p.host_plan) {
+      // the entries are already in shared memory (stage_host_plan, before
+      // the wait); a plan is only used if cu_seqlens reads {0, T}
       const bool valid = p.cu[0] == 0 && p.cu[1] == p.T;   // the same two words in every thread
-      const int n1 = valid ? hp.hdr.n_e1 : 0, n2 = valid ? hp.hdr.n_e2 : 0;
-      constexpr int kVecs = (int)(sizeof(Entry) / sizeof(uint4));
-      const uint4* h1 = reinterpret_cast<const uint4*>(hp.e1);
-      const uint4* h2 = reinterpret_cast<const uint4*>(hp.e2);
-      uint4* d1 = reinterpret_cast<uint4*>(lp->e1);
-      uint4* d2 = reinterpret_cast<uint4*>(lp->e2);
-      for (int i = threadIdx.x; i < (n1 + n2) * kVecs; i += blockDim.x) {
-        if (i < n1 * kVecs) d1[i] = h1[i];
-        else d2[i - n1 * kVecs] = h2[i - n1 * kVecs];
-      }
       if (threadIdx.x == 0) {
-        lp->seqs[0] = hp.seq;
         PlanHeader h = hp.hdr;
         if (!valid) {
           h = PlanHeader{};
