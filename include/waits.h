@@ -101,9 +101,11 @@ waits_status waits_workspace_size(const waits_shape* shape, size_t* bytes);
  * itself -- at most 32 sequences and, from a bound on the rows whose fp32
  * weight is non-zero (about b + 89/a per sequence), at most 32 planned
  * entries per pass with all active rows of a sequence in 4 Q tiles -- else
- * 3 (a planner kernel first).  Either way the results are the same.  The
- * environment variable WAITS_PLANNER_KERNEL=1 makes every call take the
- * planner kernel (a debugging aid).
+ * 4 (a planner kernel first, and between the passes a kernel that merges
+ * every row's bias once; 3, without it, under WAITS_SCORER=tc).  Either way
+ * the results are the same.  The environment variable
+ * WAITS_PLANNER_KERNEL=1 makes every call take the planner kernel (a
+ * debugging aid).
  * Host-only; touches no device state.
  * Errors: WAITS_ERR_ARG if shape or kernels is NULL, or a < 0 / non-finite,
  * or b < 0; shape errors as below.

@@ -275,6 +275,10 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
         if (js[k] >= 0) s.bias_stat[(wg + kWGs * k) * kTile + t] = bs[k];
       bar_sync(kBarAll, kEpiThreads);
     }
+    // P2K with merged biases: each streamed Q tile's row bias is loaded one
+    // step ahead, so its latency overlaps the previous step's arithmetic
+    const bool ahead = PASS == 2 && e.mode == kModeP2K && p.bias_ready && wg == 0;
+    float nb = ahead && st0 < st1 ? merged_bias(p, p.e1, si, g, e.step0 + st0, t) : 0.f;
     for (int st = st0; st < st1; ++st) {
       const int o = e.step0 + st;
       const int sb = sstep & 1;
@@ -282,10 +286,15 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
       float* bias_o = s.bias_strm + sb * kTile;
       if (PASS == 2 && e.mode == kModeP2K) {
         if (wg == 0) {
-          const int js[1] = {o};
-          float bs[1];
-          qrow_bias<1>(p, si, g, js, t, bs);
-          bias_o[t] = bs[0];
+          if (ahead) {
+            bias_o[t] = nb;
+            if (st + 1 < st1) nb = merged_bias(p, p.e1, si, g, o + 1, t);
+          } else {
+            const int js[1] = {o};
+            float bs[1];
+            qrow_bias<1>(p, si, g, js, t, bs);
+            bias_o[t] = bs[0];
+          }
         }
         bar_sync(kBarAll, kEpiThreads);
       }
@@ -548,6 +557,37 @@ cudaError_t launch_score_passes(const PassArgs& a, const HostPlan* hp, int grid,
   static const HostPlan kNone{};
   const HostPlan& h = hp ? *hp : kNone;
   return a.d == 64 ? launch_d<64>(a, h, grid, s) : launch_d<128>(a, h, grid, s);
+}
+
+// Each row's bias (log2 of its curve weight minus its log2-sum-exp) from its
+// pass-1 partials, merged once for pass 2 instead of once per stationary
+// K-tile group that streams the row: thread (entry, slot, row) runs the
+// merge pass 2 would run and writes the result over the entry's first
+// partial (it alone reads or writes those slots).
+__global__ void __launch_bounds__(256) row_bias_kernel(const __grid_constant__ PassArgs p) {
+  pdl_allow_next();
+  pdl_wait();
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t e = idx / (kMaxStat1 * kTile);
+  const int i = (int)((idx / kTile) % kMaxStat1), r = (int)(idx % kTile);
+  if (e >= p.hdr->n_e1) return;
+  const Entry en = p.e1[e];
+  if (i >= en.n_stat || en.n_units <= 0) return;
+  const SeqInfo si = p.seqs[en.seq];
+  const int js[1] = {en.stat0 + i};
+  float b[1];
+  qrow_bias<1>(p, p.e1, si, en.g, js, r, b);
+  p.part1[((size_t)en.unit_base * kMaxStat1 + i) * kTile + r] = make_float2(b[0], 0.f);
+}
+
+cudaError_t launch_row_bias(const PassArgs& a, int64_t max_e1, cudaStream_t s) {
+  const int64_t threads = max_e1 * kMaxStat1 * kTile;
+  const int64_t blocks = (threads + 255) / 256;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  PassArgs b = a;
+  b.bias_ready = 0;
+  return launch_pdl(row_bias_kernel, dim3((unsigned)blocks), dim3(256), 0, s, b);
 }
 
 cudaError_t launch_score_pass2(const PassArgs& a, int grid, cudaStream_t s) {

@@ -265,9 +265,22 @@ __device__ inline float2 lse_merge(float2 x, float2 y) {
 // the keys, from the pass-1 partials of the row's units.  The partials of
 // all NR rows are loaded together (kMergeBatch units per row in flight) and
 // merged in unit order as a maximum, then a sum of the rescaled partial sums.
+// Row r's bias of Q tile j, already merged by row_bias_kernel: one load.
+__device__ inline float merged_bias(const PassArgs& p, const Entry* e1, const SeqInfo& si, int g,
+                                    int j, int r) {
+  const int ngrp = (si.nqt + kMaxStat1 - 1) / kMaxStat1;
+  const Entry& e = e1[si.e1 + g * ngrp + j / kMaxStat1];
+  return __ldcg(&p.part1[((size_t)e.unit_base * kMaxStat1 + j % kMaxStat1) * kTile + r].x);
+}
+
 template <int NR>
 __device__ inline void qrow_bias(const PassArgs& p, const Entry* e1, const SeqInfo& si, int g,
                                  const int (&j)[NR], int r, float (&out)[NR]) {
+  if (p.bias_ready) {
+#pragma unroll
+    for (int k = 0; k < NR; ++k) out[k] = j[k] >= 0 ? merged_bias(p, e1, si, g, j[k], r) : -INFINITY;
+    return;
+  }
   if (p.lse) {
     // the caller's natural-log row LSE replaces pass 1: log2 w - lse * log2(e)
     constexpr float kLog2e = 1.4426950408889634f;

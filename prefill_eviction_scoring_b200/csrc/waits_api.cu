@@ -206,8 +206,12 @@ waits_status enqueue_score(const waits_shape* s, const void* Q, const void* K, f
     err = launch_sparse_passes(p, p.host_plan ? &hp : nullptr, grid, st);
   else if (lse)
     err = launch_score_passes(p, nullptr, grid, st);   // pass 2 only
-  else if ((err = launch_sparse_pass1(p, grid, st)) == cudaSuccess)
-    err = launch_score_pass2(p, grid, st);
+  else if ((err = launch_sparse_pass1(p, grid, st)) == cudaSuccess &&
+           (err = launch_row_bias(p, L.max_e1, st)) == cudaSuccess) {
+    PassArgs p2 = p;
+    p2.bias_ready = 1;   // pass 2 reads the merged row biases
+    err = launch_score_pass2(p2, grid, st);
+  }
   if (err != cudaSuccess) return cuda_fail("scorer launch", err);
   return WAITS_OK;
 }
@@ -281,7 +285,7 @@ waits_status waits_score_kernels(const waits_shape* shape, float a, int32_t b,
   if (!kernels || !std::isfinite(a) || a < 0.0f || b < 0) return WAITS_ERR_ARG;
   const waits_status st = check_shape(shape);
   if (st != WAITS_OK) return st;
-  *kernels = local_plan_fits(shape, a, b) ? 2 : 3;
+  *kernels = local_plan_fits(shape, a, b) ? 2 : (force_tc_scorer() ? 3 : 4);
   return WAITS_OK;
 }
 

@@ -251,6 +251,9 @@ struct PassArgs {
   // natural-log row LSE [Hq, T] given by the caller (waits_score_with_lse):
   // pass 1 is not run and pass 2 takes its row biases from it; else null
   const float* lse;
+  // 1: every pass-1 entry's merged row biases sit in the first unit's
+  // partial slots (bias in .x; row_bias_kernel ran after pass 1)
+  int bias_ready;
   // limit of every bounded wait in the main loops (ns); testing aid: with
   // withhold_mma the MMA warp issues nothing, so those waits run out
   uint64_t wait_ns;
@@ -321,6 +324,9 @@ cudaError_t launch_sparse_passes(const PassArgs& a, const HostPlan* hp, int grid
 // 256-column kernel (bit-identical row partials), pass 2 by score_tc.cu's.
 cudaError_t launch_sparse_pass1(const PassArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_score_pass2(const PassArgs& a, int grid, cudaStream_t s);
+// Between the passes of a planner-kernel plan: every row's bias, merged
+// once from its pass-1 partials (max_e1 bounds the plan's pass-1 entries).
+cudaError_t launch_row_bias(const PassArgs& a, int64_t max_e1, cudaStream_t s);
 cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
 // K == nullptr: selection only; else also the compaction of K and V into
 // Ko, Vo (the rows of the kept positions, zeros past kept_len).

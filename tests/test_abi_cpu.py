@@ -170,21 +170,25 @@ def _kernels(lib, shape, a, b):
     return st, n.value
 
 
-def test_score_kernel_count(lib):
+def test_score_kernel_count(lib, monkeypatch):
     """Small plans are rebuilt inside the scorer (2 kernels); large ones take
-    the planner kernel first (3)."""
+    the planner kernel first and merge the row biases between the passes (4;
+    3 with the general kernel forced for both passes)."""
+    monkeypatch.delenv("WAITS_SCORER", raising=False)
     llama8b = _shape(total_tokens=32768, max_seqlen=32768)
     assert _kernels(lib, llama8b, 1.0, 16) == (0, 2)     # ~105 active rows: 4 Q tiles
     assert _kernels(lib, llama8b, 10.0, 1) == (0, 2)
-    assert _kernels(lib, llama8b, 0.0, 16) == (0, 3)     # every row active
-    assert _kernels(lib, llama8b, 0.01, 128) == (0, 3)   # ~9000 active rows
+    assert _kernels(lib, llama8b, 0.0, 16) == (0, 4)     # every row active
+    assert _kernels(lib, llama8b, 0.01, 128) == (0, 4)   # ~9000 active rows
     batch = _shape(nseq=40, total_tokens=40 * 512, max_seqlen=512, num_kv_heads=4,
                    num_q_heads=28)
-    assert _kernels(lib, batch, 1.0, 16) == (0, 3)        # more than 32 sequences
+    assert _kernels(lib, batch, 1.0, 16) == (0, 4)        # more than 32 sequences
     two = _shape(nseq=2, total_tokens=2 * 8192, max_seqlen=8192)
     assert _kernels(lib, two, 1.0, 16) == (0, 2)          # 8 heads x 2 x 2 = 32 pass-1 entries
     three = _shape(nseq=3, total_tokens=3 * 8192, max_seqlen=8192)
-    assert _kernels(lib, three, 1.0, 16) == (0, 3)        # 48 pass-1 entries
+    assert _kernels(lib, three, 1.0, 16) == (0, 4)        # 48 pass-1 entries
+    monkeypatch.setenv("WAITS_SCORER", "tc")
+    assert _kernels(lib, three, 1.0, 16) == (0, 3)        # general kernel, no bias merge
     assert _kernels(lib, llama8b, -1.0, 16)[0] == 1
     assert _kernels(lib, llama8b, 1.0, -1)[0] == 1
     assert lib.waits_score_kernels(ctypes.byref(llama8b), 1.0, 16, None) == 1

@@ -145,7 +145,7 @@ def test_in_cta_plan_equals_planner_kernel(make, a, b, monkeypatch):
     monkeypatch.setenv("WAITS_DEVICE_PLAN", "1")
     s_device = api.score(lay.Q, lay.K, lay.cu_seqlens, sigmoid_a=a, window=b).clone()
     monkeypatch.setenv("WAITS_PLANNER_KERNEL", "1")
-    assert kernels() == 3
+    assert kernels() == 4
     s_kernel = api.score(lay.Q, lay.K, lay.cu_seqlens, sigmoid_a=a, window=b)
     torch.cuda.synchronize()
     assert torch.equal(s_local.view(torch.int32), s_device.view(torch.int32))
