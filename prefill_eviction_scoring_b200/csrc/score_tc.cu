@@ -275,28 +275,31 @@ __device__ void epilogue(const PassArgs& p, const Smem& s, const Entry* E, UnitI
         if (js[k] >= 0) s.bias_stat[(wg + kWGs * k) * kTile + t] = bs[k];
       bar_sync(kBarAll, kEpiThreads);
     }
-    // P2K with merged biases: each streamed Q tile's row bias is loaded one
-    // step ahead, so its latency overlaps the previous step's arithmetic
-    const bool ahead = PASS == 2 && e.mode == kModeP2K && p.bias_ready && wg == 0;
+    // P2K with merged biases: each warpgroup loads each streamed Q tile's
+    // row biases itself, one step ahead (the latency overlaps the previous
+    // step's arithmetic), into its own buffers, so the groups do not wait
+    // for each other at every step
+    const bool ahead = PASS == 2 && e.mode == kModeP2K && p.bias_ready;
     float nb = ahead && st0 < st1 ? merged_bias(p, p.e1, si, g, e.step0 + st0, t) : 0.f;
     for (int st = st0; st < st1; ++st) {
       const int o = e.step0 + st;
       const int sb = sstep & 1;
       ++sstep;
-      float* bias_o = s.bias_strm + sb * kTile;
+      float* bias_o = s.bias_strm + (ahead ? wg * 2 + sb : sb) * kTile;
       if (PASS == 2 && e.mode == kModeP2K) {
-        if (wg == 0) {
-          if (ahead) {
-            bias_o[t] = nb;
-            if (st + 1 < st1) nb = merged_bias(p, p.e1, si, g, o + 1, t);
-          } else {
+        if (ahead) {
+          bias_o[t] = nb;
+          if (st + 1 < st1) nb = merged_bias(p, p.e1, si, g, o + 1, t);
+          bar_sync(1 + wg, 128);
+        } else {
+          if (wg == 0) {
             const int js[1] = {o};
             float bs[1];
             qrow_bias<1>(p, si, g, js, t, bs);
             bias_o[t] = bs[0];
           }
+          bar_sync(kBarAll, kEpiThreads);
         }
-        bar_sync(kBarAll, kEpiThreads);
       }
       float col = 0.f;
 #pragma unroll
