@@ -52,8 +52,8 @@ L2_BYTES = 126 << 20
 # (N = 32768, a = 1, b = 16) from the committed ncu capture of the sparse
 # scorer (both passes).  Valid only for the scorer sources it was taken on
 # (sha256 of score_sparse.cu followed by scorer_common.cuh).
-PROFILED_SCORER = {"sha256_prefix": "3373f1a0c625257c",
-                   "dram_bytes": 68_217_856 + 2_074_624 + 68_379_136 + 1_420_544}
+PROFILED_SCORER = {"sha256_prefix": "f209460cda5c7ebf",
+                   "dram_bytes": 68_249_856 + 2_073_856 + 68_376_064 + 1_140_992}
 PROFILED_SOURCES = ("score_sparse.cu", "scorer_common.cuh")
 
 
