@@ -50,9 +50,10 @@ MUFU_EX2_PER_CLK_PER_SM = 16   # sm_100: 4 SFU lanes per SM sub-partition x 4
 L2_BYTES = 126 << 20
 # DRAM bytes (read + write) of one waits_score call on one 8B-shaped layer
 # (N = 32768, a = 1, b = 16) from the committed ncu capture of the sparse
-# scorer (both passes).  Valid only for the scorer sources it was taken on
-# (sha256 of score_sparse.cu followed by scorer_common.cuh).
-PROFILED_SCORER = {"sha256_prefix": "f209460cda5c7ebf",
+# scorer (both passes).  Valid only for the scorer code it was taken on
+# (scorer_source_hash: score_sparse.cu and scorer_common.cuh, comments left
+# out).
+PROFILED_SCORER = {"sha256_prefix": "bdc00e2d01d32005",
                    "dram_bytes": 68_249_856 + 2_073_856 + 68_376_064 + 1_140_992}
 PROFILED_SOURCES = ("score_sparse.cu", "scorer_common.cuh")
 
@@ -240,13 +241,25 @@ def rooflines(lens, Hq, Hkv, d, a, b, B, t_score_ms, t_sc_ms, layer_ms, pk, sm_c
     return head, other
 
 
+def code_only(text: str) -> str:
+    """A C++/CUDA source without its comments and with whitespace runs
+    collapsed: what the compiler sees of it (no string literal in the hashed
+    files holds a comment marker)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def scorer_source_hash() -> str:
-    """sha256 of the sparse scorer's sources, in PROFILED_SOURCES order."""
+    """sha256 of the sparse scorer's code (comments and layout left out), in
+    PROFILED_SOURCES order: a comment-only edit keeps the profiled counters."""
     import hashlib
     h = hashlib.sha256()
     for name in PROFILED_SOURCES:
-        with open(os.path.join(ROOT, "prefill_eviction_scoring_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "prefill_eviction_scoring_b200", "csrc", name)) as f:
+            h.update(code_only(f.read()).encode())
+            h.update(b"\0")
     return h.hexdigest()
 
 

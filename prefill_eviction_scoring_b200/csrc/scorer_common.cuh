@@ -68,9 +68,9 @@ __device__ inline float hsum8(const float2 (&a)[4]) {
 // Column pairs whose exponential runs on the FMA pipe instead of the MUFU
 // (which does 16 ex2 per clock per SM and bounds the unmasked passes): bit
 // (pair index mod 8) of this mask.  Three in eight measured best with the
-// shift-add exponential below (an epilogue-only loop over TMEM tiles: pass 1
-// 885 clocks per 128x128 tile against 1096 with the MUFU alone, pass 2 865;
-// two in eight 995 / 905, four in eight 951 / 906).
+// shift-add exponential below (an epilogue-only loop over TMEM tiles, clocks
+// per 128x128 tile: pass 1 885 against 1096 with the MUFU alone, 995 with two
+// in eight, 951 with four; pass 2 865, 906 with four, 999 with five).
 constexpr uint32_t kPolyPairs = 0x92u;
 __device__ constexpr bool poly_col(int c) { return (kPolyPairs >> ((c >> 1) & 7)) & 1u; }
 

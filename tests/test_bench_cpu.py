@@ -107,3 +107,16 @@ def test_cases_cover_every_configuration():
     sweep = bench.selected_cases(bench.parse(["--config", "all"]))
     assert {c.B for c in sweep if c.name == "llama8b"} == {128, 512, 2048}
     assert [c.B for c in bench.selected_cases(bench.parse([]))] == [2048]
+
+
+def test_scorer_hash_ignores_comments_only():
+    """The profiled-traffic key changes with the scorer's code, not with its
+    comments or layout."""
+    import bench
+    a = "int f(int x) { // one\n  return x + 1; /* two\n lines */ }\n"
+    b = "int f(int x)\n{\n  return x + 1;\n}"
+    c = "int f(int x) { return x + 2; }"
+    assert bench.code_only(a) == bench.code_only(b)
+    assert bench.code_only(a) != bench.code_only(c)
+    assert bench.profiled_traffic(bench.Case("llama8b", "llama8b", 1.0, 16, 16, 2048, 32)) \
+        == bench.PROFILED_SCORER["dram_bytes"]
