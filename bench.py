@@ -54,7 +54,7 @@ L2_BYTES = 126 << 20
 # (scorer_source_hash: score_sparse.cu and scorer_common.cuh, comments left
 # out).
 PROFILED_SCORER = {"sha256_prefix": "bdc00e2d01d32005",
-                   "dram_bytes": 68_249_856 + 2_073_856 + 68_376_064 + 1_140_992}
+                   "dram_bytes": 68_235_264 + 1_709_312 + 68_376_576 + 1_453_056}
 PROFILED_SOURCES = ("score_sparse.cu", "scorer_common.cuh")
 
 
